@@ -1,0 +1,429 @@
+#!/usr/bin/env python3
+"""Benchmark of the RAT+ sequence-mixer hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  prefill of the long-context layer (B=2, T=16384, H=16, Dh=128, D=64, W=128):
+    fused key/value scan + dilated/windowed attention;
+  decode burst of the decode-from-32K-context workload (B=64, H=16, D=64,
+    W=128): 256 fused decode steps (recurrence step, cache append, split-K
+    attention over the D-compressed cache), captured in one CUDA graph.
+`value` is prefill tokens/s of the T=16K, D=64 layer (whole job, all ranks);
+decode tokens/s is reported beside it.  Kernels are timed with CUDA events on
+the stream they are launched on; multi-GPU runs are weak-scaled replicas (no
+data-path collective) timed as the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only executable statement of
+the method there is) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PREFILL = "bf16_long_T16384_D64_W128"
+DECODE = "bf16_decode_ctx32768_D64_W128"
+METRIC = "RAT+ layer prefill & decode tokens/s at T=16K, D=64; % of HBM/tensor roofline"
+
+
+# ----------------------------------------------------------------------------- counts
+def attention_pairs(T, D, W, dense=False):
+    """Exact number of (query, key) pairs of one (b, h): sum_t |K(t)|."""
+    t = np.arange(T, dtype=np.int64)
+    if dense or D == 1:
+        return int((t + 1).sum())
+    if W <= 0:
+        return int((t // D + 1).sum())
+    lo = np.maximum(0, t - W + 1)
+    F = lambda x: np.where(x >= 0, (x + 1) // D, 0)     # #{0 <= j <= x : j mod D = D-1}
+    dup = F(t - 1) - F(lo - 1)
+    return int((t // D + np.minimum(W, t + 1) - dup).sum())
+
+
+def prefill_counts(w):
+    E = w.B * w.T * w.H * w.Dh
+    pairs = 0
+    for h in range(w.H):
+        pairs += w.B * attention_pairs(w.T, w.D, w.W, dense=h in w.dense_heads)
+    return {
+        "scan_bytes": 5 * E * 2,                  # read xk, xv, g; write hk, hv (bf16)
+        "attn_bytes": 4 * E * 2,                  # read q, hk, hv; write o
+        "attn_flops": 4 * w.Dh * pairs,           # QK^T + PV over the key sets
+        "pairs": pairs,
+    }
+
+
+def decode_bytes_per_step(w, t):
+    """Algorithmic HBM bytes of one decode token for every (b, h) at position t."""
+    total = 0
+    for h in range(w.H):
+        Dd = 1 if h in w.dense_heads else w.D
+        n_slots = t // Dd
+        n_win = 0
+        if w.W > 0 and Dd > 1:
+            lo = max(0, t - w.W + 1)
+            n_win = sum(1 for p in range(lo, t) if p % Dd != Dd - 1)
+        rows = n_slots + n_win
+        per = rows * 2 * w.Dh * 2                 # K and V rows read
+        per += 2 * w.Dh * 4 * 2                   # fp32 state read + write (k, v)
+        per += 4 * w.Dh * 2 + w.Dh * 2            # q, xk, xv, g read; o written
+        per += (2 * w.Dh * 2) if w.W > 0 else 0   # ring write
+        per += (2 * w.Dh * 2) if t % Dd == Dd - 1 else 0   # dilated append
+        total += w.B * per
+    return total
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (clocks and throttle reasons)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_sample(seconds_target=12.0):
+    """Time the fp64 oracle on a bounded sample of the prefill workload.
+
+    Sample: the scan of both streams over the first `ts` tokens of every
+    sequence (all channels), and attention for `nr` random query rows (b, t, h)
+    of the full-length layer.  Tokens/s = 1 / (scan s/token + attention s/token)
+    where one token is one position of all H heads.
+    """
+    import oracle
+    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
+    w = WORKLOADS[PREFILL]
+    oracle.build()
+    ts = 1024
+    q, xk, xv, g = prefill_inputs(w.B, ts, w.H, w.Dh, w.dtype, w.gate_mean, w.gate_std, seed=0)
+    x64k, x64v, g64 = (x.to(torch.float64).numpy() for x in (xk, xv, g))
+    t0 = time.perf_counter()
+    oracle.scan(x64k, g64)
+    oracle.scan(x64v, g64)
+    t_scan = (time.perf_counter() - t0) / (w.B * ts)
+    # attention rows: queries from the full-length key sets; keys drawn N(0, 1)
+    rng = np.random.default_rng(0)
+    nr = 2048
+    heads = [0]
+    Tfull = w.T
+    qf, kf, vf, _ = prefill_inputs(1, Tfull, 1, w.Dh, w.dtype, seed=1)
+    rows = np.stack([np.zeros(nr, np.int64), rng.integers(0, Tfull, nr), np.zeros(nr, np.int64)], 1)
+    q64, k64, v64 = (x.to(torch.float64).numpy() for x in (qf, kf, vf))
+    t0 = time.perf_counter()
+    oracle.attention(q64, k64, v64, w.D, w.W, rows=rows)
+    t_attn_row = (time.perf_counter() - t0) / nr
+    t_attn = t_attn_row * w.H
+    tok_s = 1.0 / (t_scan + t_attn)
+    return {"value": tok_s, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "fp64 oracle: scan of both streams over %d tokens x %d sequences (all %d "
+                      "channels) + attention of %d random query rows of one head at T=%d, D=%d, "
+                      "W=%d; per-token cost = scan + %d heads x row cost" % (
+                          ts, w.B, w.H * w.Dh, nr, Tfull, w.D, w.W, w.H),
+            "scan_s_per_token": t_scan, "attn_s_per_token": t_attn}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS
+    w = WORKLOADS[PREFILL]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        r = oracle_sample()
+        if i >= args.warmup:
+            vals.append(r)
+    v = statistics.median([r["value"] for r in vals])
+    tokens = w.B * w.T
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tokens / v * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": PREFILL, "B": w.B, "T": w.T, "H": w.H, "Dh": w.Dh, "D": w.D,
+                   "W": w.W},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
+                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, rank, world, local_rank):
+    import recurrence_augmented_dilated_chunked_b200 as ratp
+    from recurrence_augmented_dilated_chunked_b200 import (WORKLOADS, decode_context,
+                                                           decode_inputs, prefill_inputs)
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    ratp.load_library()
+    stream = torch.cuda.current_stream(dev)
+    wp, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
+
+    # ---- prefill inputs (seeded, synthetic; a different seed per rank) ----
+    q, xk, xv, g = prefill_inputs(wp.B, wp.T, wp.H, wp.Dh, wp.dtype, wp.gate_mean, wp.gate_std,
+                                  seed=rank)
+    q_h, xk_h, xv_h, g_h = (t.pin_memory() for t in (q, xk, xv, g))
+    qd, xkd, xvd, gd = (t.to(dev) for t in (q_h, xk_h, xv_h, g_h))
+    hk, hv, o = (torch.empty_like(qd) for _ in range(3))
+    ws = ratp.scan_workspace(wp.B, wp.T, wp.H, wp.Dh, qd.dtype, dev)
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+
+    # ---- decode context + per-step inputs ----
+    steps = wd.decode_steps
+    T_max = wd.decode_ctx + steps
+    kd, vd, kw, vw, st0 = decode_context(wd.B, wd.H, wd.Dh, wd.decode_ctx, wd.D, wd.W, seed=2 + rank)
+    dq, dxk, dxv, dg = (t.to(dev) for t in decode_inputs(steps, wd.B, wd.H, wd.Dh, "bf16",
+                                                         wd.gate_mean, wd.gate_std, seed=1 + rank))
+    cache = ratp.KVCache(wd.B, wd.H, wd.Dh, T_max, wd.D, wd.W)
+    kc, vc = cache.dil_rows("k"), cache.dil_rows("v")
+    for h in range(wd.H):
+        off, _ = cache.head_rows(h)
+        n = kd[h].shape[1]
+        kc[:, off:off + n] = kd[h].to(dev)
+        vc[:, off:off + n] = vd[h].to(dev)
+    cache.ring("k").copy_(kw.to(dev))
+    cache.ring("v").copy_(vw.to(dev))
+    state0 = st0.to(dev)
+    state = state0.clone()
+    dout = torch.empty(steps, wd.B, wd.H, wd.Dh, dtype=torch.bfloat16, device=dev)
+    lens = cache.lengths()
+
+    def decode_burst():
+        lens.fill_(wd.decode_ctx)
+        for i in range(steps):
+            cache.decode_step(dq[i], dxk[i], dxv[i], dg[i], state, out=dout[i])
+
+    # capture the 256-step burst once (warm the kernels first)
+    decode_burst()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        decode_burst()
+    torch.cuda.synchronize()
+    ratp.last_error(dev)
+
+    def prefill(ev=None):
+        if ev:
+            ev[0].record(stream)
+        ratp.scan_prefill_kv(xkd, xvd, gd, hk=hk, hv=hv, workspace=ws)
+        if ev:
+            ev[1].record(stream)
+        ratp.dilated_attn_prefill(qd, hk, hv, wp.D, wp.W, out=o)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        prefill()
+        graph.replay()
+    torch.cuda.synchronize()
+    ratp.last_error(dev)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            prefill(evs[i])
+            graph.replay()
+            evs[i][3].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    ratp.last_error(dev)
+    scan_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    dec_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+
+    # ---- end to end through the public API with host buffers ----
+    e_evs = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    for i in range(args.warmup + args.steps):
+        if i == args.warmup:
+            torch.cuda.synchronize()
+            e_evs[0].record(stream)
+        for src, dst in ((q_h, qd), (xk_h, xkd), (xv_h, xvd), (g_h, gd)):
+            dst.copy_(src, non_blocking=True)
+        prefill()
+        o_h.copy_(o, non_blocking=True)
+    e_evs[1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e_evs[0].elapsed_time(e_evs[1])
+    ratp.last_error(dev)
+
+    # ---- max over ranks ----
+    def rmax(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    s_scan, s_attn, s_dec = rmax(sum(scan_ms)), rmax(sum(attn_ms)), rmax(sum(dec_ms))
+    s_total, s_e2e = rmax(total_ms), rmax(e2e_ms)
+    if rank != 0:
+        return 0
+
+    K = args.steps
+    pc = prefill_counts(wp)
+    peaks = measured_peaks()
+    prefill_tokens = wp.B * wp.T
+    prefill_s = (s_scan + s_attn) / 1e3
+    value = world * prefill_tokens * K / prefill_s
+    decode_tok_s = world * wd.B * steps * K / (s_dec / 1e3)
+    scan_gbs = pc["scan_bytes"] * K / (s_scan / 1e3) / 1e9
+    attn_gbs = pc["attn_bytes"] * K / (s_attn / 1e3) / 1e9
+    attn_tfs = pc["attn_flops"] * K / (s_attn / 1e3) / 1e12
+    dec_bytes = sum(decode_bytes_per_step(wd, wd.decode_ctx + i) for i in range(steps))
+    dec_gbs = dec_bytes * K / (s_dec / 1e3) / 1e9
+    kernels = {
+        "scan_kv": {"ms_per_launch": s_scan / K, "achieved_gbs": scan_gbs,
+                    "frac_hbm": scan_gbs / peaks["hbm_gbs"], "alg_bytes": pc["scan_bytes"]},
+        "dilated_attn": {"ms_per_launch": s_attn / K, "achieved_gbs": attn_gbs,
+                         "frac_hbm": attn_gbs / peaks["hbm_gbs"], "achieved_tflops": attn_tfs,
+                         "frac_tensor": attn_tfs / peaks["bf16_tflops"], "alg_bytes": pc["attn_bytes"],
+                         "alg_flops": pc["attn_flops"]},
+        "decode_step": {"ms_per_launch": s_dec / K / steps, "achieved_gbs": dec_gbs,
+                        "frac_hbm": dec_gbs / peaks["hbm_gbs"], "alg_bytes_per_launch": dec_bytes / steps},
+    }
+    # dominant kernel of the timed step by share of device time
+    shares = {"scan_kv": s_scan, "dilated_attn": s_attn, "decode_step": s_dec}
+    dom = max(shares, key=shares.get)
+    kd_ = kernels[dom]
+    roof = {"kernel": dom, "bound": "hbm", "achieved": kd_["achieved_gbs"], "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": kd_["frac_hbm"], "traffic": None,
+            "peak_source": peaks["source"]}
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, xk_h, xv_h, g_h))
+    d2h = o_h.numel() * o_h.element_size()
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": s_total / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": PREFILL, "B": wp.B, "T": wp.T, "H": wp.H, "Dh": wp.Dh, "D": wp.D,
+                   "W": wp.W, "decode_workload": DECODE, "decode_B": wd.B,
+                   "decode_ctx": wd.decode_ctx, "decode_steps": steps,
+                   "l2": "no flush: every step streams > 1 GB (inputs larger than L2)",
+                   "parallelism": "replicas x%d" % world},
+        "prefill": {"tokens_per_s": value, "ms": (s_scan + s_attn) / K},
+        "decode": {"tokens_per_s": decode_tok_s, "ms_per_token_step": s_dec / K / steps,
+                   "graph": "256 decode launches per CUDA graph"},
+        "kernels": kernels,
+        "roofline": roof,
+        "e2e": {"value": world * prefill_tokens * args.steps / (s_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "prefill through the C ABI from pinned host q/xk/xv/g to host o"},
+        "gpu_launches": K * (2 + steps),
+        "clocks": clk.summary(),
+        "wall_s": t_wall,
+    }
+    if not args.no_cpu_baseline and world >= 1:
+        line["cpu_baseline"] = oracle_sample()
+    print(json.dumps(line), flush=True)
+    del graph
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        if args.impl == "reference":
+            return run_reference(args, rank, world)
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1 and args.impl == "ours":
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,193 @@
+/*
+ * ratp.h -- C ABI of the B200 (sm_100a) RAT+ sequence-mixer library.
+ *
+ * The library computes the data-parallel hot path of RAT+ ("RAT+: Train
+ * Dense, Infer Sparse -- Recurrence Augmented Attention for Dilated
+ * Inference", arXiv 2602.18196):
+ *
+ *   1. the full-sequence forget-gate recurrence over the key and value
+ *      streams, h_t = g_t * h_{t-1} + (1 - g_t) * x_t per channel, h_{-1} = 0
+ *      (zhichai.net write-up "RAT+ 深度拆解", section 2.1: forget-gate
+ *      recurrence over the whole sequence, parallel associative scan at
+ *      prefill);
+ *   2. causal softmax attention of query t over the recurrent keys/values at
+ *      S_D(t) = { j < t : j mod D = D-1 } U { t }, optionally united with the
+ *      window { j : t-W < j <= t } (RAT+ abstract: dilated attention of
+ *      dilation D cuts attention FLOPs and the KV cache by D, optionally with
+ *      local windows; write-up section 1);
+ *   3. head-wise hybrids: heads flagged in head_mask run dense (D = 1)
+ *      (write-up section 6: the first heads dense, the rest dilated).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are dense, row-major, on the current CUDA device, and owned by
+ *     the caller.  Prefill tensors are [B][T][H][Dh]; decode tensors are
+ *     [B][H][Dh].  Every device pointer must be 16-byte aligned.
+ *   - dtype is RATP_F32 or RATP_BF16 for all tensor arguments of one call
+ *     (recurrent state and final states are always fp32).  Arithmetic is fp32.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     stream-ordered and asynchronous; none synchronises the host except
+ *     ratp_last_error().
+ *   - Return value: RATP_OK (0) or a ratp_status code.  Argument errors are
+ *     detected on the host before any launch and leave outputs untouched.
+ *     Asynchronous device-side errors (a bounded wait that ran out, a cache
+ *     append beyond capacity) are recorded in a per-device error word that
+ *     ratp_last_error() returns.  The library never aborts the process.
+ *   - The library allocates no device memory.  Scratch space is passed in by
+ *     the caller (sizes from the *_bytes queries).
+ */
+#ifndef RATP_H_
+#define RATP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ratp_status {
+  RATP_OK = 0,
+  RATP_ERR_ARG = 1,         /* null pointer, negative size, bad enum */
+  RATP_ERR_SHAPE = 2,       /* unsupported shape (Dh, H, sizes)        */
+  RATP_ERR_ALIGN = 3,       /* pointer not 16-byte aligned            */
+  RATP_ERR_CAPACITY = 4,    /* workspace/cache too small, cache full  */
+  RATP_ERR_TIMEOUT = 5,     /* a bounded device wait ran out          */
+  RATP_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed      */
+  RATP_ERR_UNSUPPORTED = 7  /* dtype/shape combination not built      */
+} ratp_status;
+
+typedef enum ratp_dtype { RATP_F32 = 0, RATP_BF16 = 1 } ratp_dtype;
+
+/* Largest head count accepted by head_mask-taking calls. */
+#define RATP_MAX_HEADS 256
+
+/* Human-readable name of a status code (static string). */
+const char* ratp_status_string(int status);
+
+/* Reads and clears the device error word of the current device after
+ * synchronising `stream`.  Returns RATP_OK or the lowest-numbered error
+ * recorded by any kernel since the previous call. */
+int ratp_last_error(void* stream);
+
+/* Number of SMs of the current device (grid sizing). */
+int ratp_device_sm_count(int* sms);
+
+/* ------------------------------------------------------------------------
+ * Prefill recurrence (write-up section 2.1).
+ *
+ * ratp_scan_workspace_bytes: bytes of device scratch that one scan call of
+ *   this shape needs (chunk descriptors of the single-pass scan).
+ * ratp_scan_prefill: h = scan(x, g) over T for every (b, channel);
+ *   x, g, h: [B][T][H][Dh] of dtype.  final_state (nullable): fp32 [B][H][Dh],
+ *   receives h_{T-1} in fp32.
+ * ratp_scan_prefill_kv: the key and value streams in one pass with one gate
+ *   tensor (g is read once): hk = scan(xk, g), hv = scan(xv, g).
+ *   final_state (nullable): fp32 [2][B][H][Dh] (k then v) -- the layout of the
+ *   decode state.
+ * workspace: device scratch of at least ratp_scan_workspace_bytes; it is
+ *   re-initialised on `stream` by every call, so calls sharing one workspace
+ *   must be ordered on one stream.  h may alias x (in-place) only when
+ *   T == 1.  Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of
+ *   64), ALIGN, CAPACITY (workspace too small).  T == 0 or B == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+int ratp_scan_workspace_bytes(int B, int T, int H, int Dh, int dtype, size_t* bytes);
+int ratp_scan_prefill(const void* x, const void* g, void* h, float* final_state,
+                      int B, int T, int H, int Dh, int dtype,
+                      void* workspace, size_t workspace_bytes, void* stream);
+int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
+                         void* hk, void* hv, float* final_state,
+                         int B, int T, int H, int Dh, int dtype,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Dilated (+ windowed) prefill attention (RAT+ abstract; write-up sections 1
+ * and 6).
+ *
+ * o[b][t][h] = sum_{j in K_h(t)} softmax_j(q[b][t][h] . hk[b][j][h] / sqrt(Dh))
+ *              * hv[b][j][h]
+ * K_h(t) = { j < t : j mod D_h = D_h-1 } U { t } U { j : t-W < j <= t }
+ * (each key once), D_h = 1 where head_mask[h] != 0, else D.
+ *
+ * q, hk, hv, o: [B][T][H][Dh] of dtype.  D >= 1, W >= 0 (0 = no window).
+ * head_mask: HOST array of H bytes, or NULL (no dense heads).
+ * ratp_dilated_attn_prefill dispatches bf16 with Dh == 128 to the tensor-core
+ * kernel (TMA + tcgen05.mma, accumulators in tensor memory) and every other
+ * supported case (fp32; Dh 64) to the CUDA-core kernel.
+ * ratp_dilated_attn_prefill_simt always runs the CUDA-core kernel
+ * (fp32 or bf16, Dh in {64, 128}).
+ * Errors: ARG, SHAPE (Dh not 64/128, H > RATP_MAX_HEADS), ALIGN, CUDA.
+ * ---------------------------------------------------------------------- */
+int ratp_dilated_attn_prefill(const void* q, const void* hk, const void* hv, void* o,
+                              int B, int T, int H, int Dh, int D, int W,
+                              const uint8_t* head_mask, int dtype, void* stream);
+int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv, void* o,
+                                   int B, int T, int H, int Dh, int D, int W,
+                                   const uint8_t* head_mask, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
+ * D-compressed KV cache and decode (RAT+ abstract: the KV cache shrinks by D).
+ *
+ * Layout (all bf16 rows of Dh elements):
+ *   Kc/Vc: dilated rows.  Head h keeps the recurrent key/value of position
+ *          p = s*D_h + D_h - 1 in slot s < cap_h = T_max / D_h.  Row of
+ *          (b, h, s) = b * rows_per_b + sum_{h' < h} cap_{h'} + s.
+ *   Kw/Vw: window ring, [B][H][W][Dh]; position p sits in row p mod W.
+ *          Absent (NULL) when W == 0.
+ *   len:   int32 [B], the number of tokens absorbed per sequence (the
+ *          position of the next token).
+ *   partial, counters: decode split-K scratch.  counters must be zero when
+ *          a decode step starts; ratp_cache_init zeroes them and every step
+ *          leaves them zero.
+ * The struct is plain data filled by ratp_cache_init; the caller owns the
+ * buffer it points into.
+ * ---------------------------------------------------------------------- */
+typedef struct ratp_cache {
+  void* Kc;
+  void* Vc;
+  void* Kw;
+  void* Vw;
+  int32_t* len;
+  float* partial;
+  uint32_t* counters;
+  int64_t rows_per_b;   /* sum_h cap_h */
+  int32_t B, H, Dh, T_max, D, W;
+  int32_t split_keys;   /* keys per decode split */
+  int32_t max_splits;   /* grid width of one decode step */
+  uint8_t dense[RATP_MAX_HEADS];
+} ratp_cache;
+
+/* Bytes of the single device buffer that holds a cache of this shape. */
+int ratp_cache_bytes(int B, int H, int Dh, int T_max, int D, int W,
+                     const uint8_t* head_mask, size_t* bytes);
+
+/* Carves `buffer` (device, >= ratp_cache_bytes) into the cache regions,
+ * fills *c, and zeroes len and the counters on `stream`.
+ * Dh must be 128 or 64, dtype is bf16.  Errors: ARG, SHAPE, ALIGN, CAPACITY. */
+int ratp_cache_init(ratp_cache* c, void* buffer, size_t bytes,
+                    int B, int H, int Dh, int T_max, int D, int W,
+                    const uint8_t* head_mask, void* stream);
+
+/* Prefill -> decode hand-off: copies the dilated rows of hk, hv (bf16
+ * [B][T][H][Dh], T <= T_max) into Kc/Vc, the last min(W, T) positions into
+ * the ring, and sets len[b] = T.  The recurrent state comes from the scan's
+ * final_state (ratp_scan_prefill_kv writes the [2][B][H][Dh] decode layout). */
+int ratp_cache_pack(ratp_cache* c, const void* hk, const void* hv, int T, void* stream);
+
+/* One decode token for every sequence (fused): state <- g*state + (1-g)*x for
+ * the key and value streams (fp32 state [2][B][H][Dh], in/out); the new
+ * recurrent key/value is appended to Kc/Vc when t mod D_h == D_h - 1 and
+ * always written to the ring; o = attention of q over the cached dilated
+ * slots s < t / D_h, the window positions t-W < p < t not among them, and the
+ * new key/value itself; len[b] += 1.
+ * q, xk, xv, g, o: bf16 [B][H][Dh].  D, W, head_mask must equal the values
+ * the cache was initialised with (ERR_ARG otherwise).  A token beyond T_max
+ * sets RATP_ERR_CAPACITY in the device error word and leaves that sequence
+ * unchanged. */
+int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* g,
+                     float* state, ratp_cache* c, void* o,
+                     int D, int W, const uint8_t* head_mask, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* RATP_H_ */

@@ -1,0 +1,282 @@
+"""ctypes binding of ``libratp.so`` (the C ABI declared in ``include/ratp.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI.  PyTorch supplies device memory and the current
+stream.  There is no CPU fallback -- if the library is missing the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libratp.so")
+MAX_HEADS = 256
+
+RATP_F32, RATP_BF16 = 0, 1
+_DTYPE = {torch.float32: RATP_F32, torch.bfloat16: RATP_BF16}
+
+STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_CAPACITY",
+          5: "ERR_TIMEOUT", 6: "ERR_CUDA", 7: "ERR_UNSUPPORTED"}
+
+
+class RatpError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__("%s failed: %s (%d)" % (fn, STATUS.get(code, "?"), code))
+
+
+class CacheStruct(ctypes.Structure):
+    """Mirror of ``struct ratp_cache``."""
+    _fields_ = [
+        ("Kc", ctypes.c_void_p), ("Vc", ctypes.c_void_p),
+        ("Kw", ctypes.c_void_p), ("Vw", ctypes.c_void_p),
+        ("len", ctypes.c_void_p), ("partial", ctypes.c_void_p), ("counters", ctypes.c_void_p),
+        ("rows_per_b", ctypes.c_int64),
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("Dh", ctypes.c_int32),
+        ("T_max", ctypes.c_int32), ("D", ctypes.c_int32), ("W", ctypes.c_int32),
+        ("split_keys", ctypes.c_int32), ("max_splits", ctypes.c_int32),
+        ("dense", ctypes.c_uint8 * MAX_HEADS),
+    ]
+
+
+_lib = None
+_lock = threading.Lock()
+
+_P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "ratp_status_string": ([_I], ctypes.c_char_p),
+    "ratp_last_error": ([_P], _I),
+    "ratp_device_sm_count": ([ctypes.POINTER(_I)], _I),
+    "ratp_scan_workspace_bytes": ([_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "ratp_scan_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
+    "ratp_scan_prefill_kv": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
+    "ratp_dilated_attn_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
+    "ratp_dilated_attn_prefill_simt": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
+    "ratp_cache_bytes": ([_I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)], _I),
+    "ratp_cache_init": ([ctypes.POINTER(CacheStruct), _P, _SZ, _I, _I, _I, _I, _I, _I, _P, _P], _I),
+    "ratp_cache_pack": ([ctypes.POINTER(CacheStruct), _P, _P, _I, _P], _I),
+    "ratp_decode_step": ([_P, _P, _P, _P, _P, ctypes.POINTER(CacheStruct), _P, _I, _I, _P, _P], _I),
+}
+
+
+def load_library(path: str = LIB_PATH):
+    """Load ``libratp.so``; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise RuntimeError(
+                    "CUDA library %s is missing; build it with "
+                    "`python -m recurrence_augmented_dilated_chunked_b200.build`" % path)
+            lib = ctypes.CDLL(path)
+            for name, (args, res) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = lib
+    return _lib
+
+
+def exported_symbols():
+    return sorted(_SIGS)
+
+
+def _check(fn, code):
+    if code != 0:
+        raise RatpError(fn, code)
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+
+
+def _mask_buf(head_mask, H):
+    if head_mask is None:
+        return None, None
+    m = bytes(1 if v else 0 for v in list(head_mask))
+    if len(m) != H:
+        raise ValueError("head_mask must have H = %d entries" % H)
+    buf = (ctypes.c_uint8 * H).from_buffer_copy(m)
+    return buf, ctypes.cast(buf, ctypes.c_void_p)
+
+
+_ws_cache = {}
+
+
+def scan_workspace(B, T, H, Dh, dtype, device) -> torch.Tensor:
+    """Device scratch for one scan call of this shape (cached per device/size)."""
+    lib = load_library()
+    n = ctypes.c_size_t()
+    _check("ratp_scan_workspace_bytes",
+           lib.ratp_scan_workspace_bytes(B, T, H, Dh, _DTYPE[dtype], ctypes.byref(n)))
+    key = (str(device), n.value)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def scan_prefill(x, g, out=None, final_state=None, workspace=None):
+    """h = forget-gate scan of x with gates g over axis 1 of [B, T, H, Dh]."""
+    lib = load_library()
+    _need(x, "x")
+    _need(g, "g", x.dtype)
+    B, T, H, Dh = x.shape
+    if out is None:
+        out = torch.empty_like(x)
+    _need(out, "out", x.dtype)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32)
+    ws = workspace if workspace is not None else scan_workspace(B, T, H, Dh, x.dtype, x.device)
+    _check("ratp_scan_prefill", lib.ratp_scan_prefill(
+        _ptr(x), _ptr(g), _ptr(out), _ptr(final_state), B, T, H, Dh, _DTYPE[x.dtype],
+        _ptr(ws), ws.numel(), _stream(x)))
+    return out
+
+
+def scan_prefill_kv(xk, xv, g, hk=None, hv=None, final_state=None, workspace=None):
+    """(hk, hv) = scans of xk and xv sharing the gate tensor g (one pass)."""
+    lib = load_library()
+    _need(xk, "xk")
+    _need(xv, "xv", xk.dtype)
+    _need(g, "g", xk.dtype)
+    B, T, H, Dh = xk.shape
+    hk = torch.empty_like(xk) if hk is None else hk
+    hv = torch.empty_like(xv) if hv is None else hv
+    _need(hk, "hk", xk.dtype)
+    _need(hv, "hv", xk.dtype)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32)
+    ws = workspace if workspace is not None else scan_workspace(B, T, H, Dh, xk.dtype, xk.device)
+    _check("ratp_scan_prefill_kv", lib.ratp_scan_prefill_kv(
+        _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(final_state),
+        B, T, H, Dh, _DTYPE[xk.dtype], _ptr(ws), ws.numel(), _stream(xk)))
+    return hk, hv
+
+
+def _attn(fn_name, q, hk, hv, D, W, head_mask, out):
+    lib = load_library()
+    _need(q, "q")
+    _need(hk, "hk", q.dtype)
+    _need(hv, "hv", q.dtype)
+    B, T, H, Dh = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.dtype)
+    _buf, mp = _mask_buf(head_mask, H)
+    _check(fn_name, getattr(lib, fn_name)(
+        _ptr(q), _ptr(hk), _ptr(hv), _ptr(out), B, T, H, Dh, int(D), int(W), mp,
+        _DTYPE[q.dtype], _stream(q)))
+    return out
+
+
+def dilated_attn_prefill(q, hk, hv, D, W=0, head_mask=None, out=None):
+    """Dilated (+ windowed) causal attention of q over recurrent hk, hv."""
+    return _attn("ratp_dilated_attn_prefill", q, hk, hv, D, W, head_mask, out)
+
+
+def dilated_attn_prefill_simt(q, hk, hv, D, W=0, head_mask=None, out=None):
+    """Same operation on the CUDA-core kernel (fp32/bf16, Dh 64/128)."""
+    return _attn("ratp_dilated_attn_prefill_simt", q, hk, hv, D, W, head_mask, out)
+
+
+def last_error(device=None):
+    """Synchronise and raise if any kernel recorded a device-side error."""
+    lib = load_library()
+    dev = torch.device("cuda" if device is None else device)
+    s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    _check("ratp_last_error", lib.ratp_last_error(s))
+
+
+def sm_count() -> int:
+    n = ctypes.c_int()
+    _check("ratp_device_sm_count", load_library().ratp_device_sm_count(ctypes.byref(n)))
+    return n.value
+
+
+class KVCache:
+    """D-compressed KV cache for decode (one device buffer, see ``ratp.h``)."""
+
+    def __init__(self, B, H, Dh, T_max, D, W=0, head_mask=None, device="cuda"):
+        lib = load_library()
+        self.B, self.H, self.Dh, self.T_max, self.D, self.W = B, H, Dh, T_max, D, W
+        self.head_mask = [1 if v else 0 for v in head_mask] if head_mask is not None else None
+        self._mask_buf, mp = _mask_buf(self.head_mask, H)
+        n = ctypes.c_size_t()
+        _check("ratp_cache_bytes", lib.ratp_cache_bytes(B, H, Dh, T_max, D, W, mp, ctypes.byref(n)))
+        self.buffer = torch.empty(n.value, dtype=torch.uint8, device=device)
+        self.c = CacheStruct()
+        _check("ratp_cache_init", lib.ratp_cache_init(
+            ctypes.byref(self.c), _ptr(self.buffer), n.value, B, H, Dh, T_max, D, W, mp,
+            _stream(self.buffer)))
+
+    def _view(self, addr, numel, dtype):
+        off = addr - self.buffer.data_ptr()
+        esz = torch.empty((), dtype=dtype).element_size()
+        return self.buffer[off: off + numel * esz].view(dtype)
+
+    def dil_rows(self, which="k"):
+        """Kc or Vc as [B, rows_per_b, Dh] bf16 (a view of the buffer)."""
+        addr = self.c.Kc if which == "k" else self.c.Vc
+        rows = self.B * self.c.rows_per_b
+        return self._view(addr, rows * self.Dh, torch.bfloat16).view(self.B, self.c.rows_per_b, self.Dh)
+
+    def ring(self, which="k"):
+        """Kw or Vw as [B, H, W, Dh] bf16 (None when W == 0)."""
+        if self.W == 0:
+            return None
+        addr = self.c.Kw if which == "k" else self.c.Vw
+        n = self.B * self.H * self.W * self.Dh
+        return self._view(addr, n, torch.bfloat16).view(self.B, self.H, self.W, self.Dh)
+
+    def lengths(self):
+        return self._view(self.c.len, self.B, torch.int32)
+
+    def head_rows(self, h):
+        """(offset, capacity) of head h inside one batch item's dilated rows."""
+        off = 0
+        for k in range(self.H):
+            cap = self.T_max if (self.head_mask and self.head_mask[k]) else self.T_max // self.D
+            if k == h:
+                return off, cap
+            off += cap
+        raise IndexError(h)
+
+    def pack(self, hk, hv, T=None):
+        _need(hk, "hk", torch.bfloat16)
+        _need(hv, "hv", torch.bfloat16)
+        T = hk.shape[1] if T is None else T
+        _check("ratp_cache_pack", load_library().ratp_cache_pack(
+            ctypes.byref(self.c), _ptr(hk), _ptr(hv), int(T), _stream(hk)))
+
+    def decode_step(self, q, xk, xv, g, state, out=None):
+        """One token per sequence; state: fp32 [2, B, H, Dh] updated in place."""
+        for t, n in ((q, "q"), (xk, "xk"), (xv, "xv"), (g, "g")):
+            _need(t, n, torch.bfloat16)
+        _need(state, "state", torch.float32)
+        if out is None:
+            out = torch.empty_like(q)
+        _need(out, "out", torch.bfloat16)
+        _check("ratp_decode_step", load_library().ratp_decode_step(
+            _ptr(q), _ptr(xk), _ptr(xv), _ptr(g), _ptr(state), ctypes.byref(self.c), _ptr(out),
+            self.D, self.W, ctypes.cast(self._mask_buf, ctypes.c_void_p) if self._mask_buf is not None else None,
+            _stream(q)))
+        return out

@@ -1,0 +1,319 @@
+// decode.cuh -- D-compressed KV cache: prefill hand-off and the fused decode
+// step (RAT+ abstract: the KV cache shrinks by the dilation D; write-up
+// section 2.1: the recurrence is a one-step state update at decode; write-up
+// section 6: dense heads).
+//
+// Decode step for token t = len[b] of every sequence, one launch:
+//   grid (split, h, b).  The keys of (b, h) form a virtual list: the cached
+//   dilated slots s < t / D_h (Kc/Vc rows), then the raw window positions
+//   t-W < p < t (ring rows; positions with p mod D_h = D_h-1 are dilated keys
+//   already in the list and are skipped).  Split i streams keys
+//   [i*split_keys, (i+1)*split_keys) with 16-byte loads, a half-warp per key
+//   (Dh = 128) and an fp32 online softmax per half-warp.
+//   Split 0 additionally performs the recurrence step for the k and v streams
+//   (fp32 state, in place), appends the bf16-rounded new key/value to Kc/Vc
+//   when t mod D_h = D_h-1, writes it into ring row t mod W, and attends to it
+//   (the query's own key).  None of these rows is read by any CTA of the
+//   same step, so there is no intra-step race.
+//   Splits publish (m, l, acc) partials; the last split of (b, h) to finish
+//   (atomic counter) merges them and writes o.  The last CTA of the grid
+//   advances len[b].  Counters return to zero, so no per-step reset is needed.
+#pragma once
+#include "common.cuh"
+
+namespace ratp {
+namespace decode {
+
+constexpr int kThreads = 128;
+
+struct Params {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* xk;
+  const __nv_bfloat16* xv;
+  const __nv_bfloat16* g;
+  __nv_bfloat16* o;
+  float* state;                 // [2][B][H][Dh]
+  __nv_bfloat16* Kc;
+  __nv_bfloat16* Vc;
+  __nv_bfloat16* Kw;
+  __nv_bfloat16* Vw;
+  int32_t* len;
+  float* partial;               // [B][H][max_splits][Dh + 2]
+  uint32_t* counters;           // [B*H + 1]
+  long long rows_per_b;
+  int B, H, D, W, T_max, split_keys, max_splits;
+  float scale_log2;
+  unsigned long long dense_bits[RATP_MAX_HEADS / 64];
+};
+
+__device__ __forceinline__ bool is_dense(const unsigned long long* bits, int h) {
+  return (bits[h >> 6] >> (h & 63)) & 1ull;
+}
+
+// Row offset of head h inside one batch item: sum of capacities of heads < h.
+__device__ __forceinline__ long long head_offset(const unsigned long long* bits, int h,
+                                                 int T_max, int D) {
+  int nd = 0;
+  for (int w = 0; w < (h >> 6); ++w) nd += __popcll(bits[w]);
+  if (h & 63) nd += __popcll(bits[h >> 6] & ((1ull << (h & 63)) - 1ull));
+  return (long long)nd * T_max + (long long)(h - nd) * (T_max / D);
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kThreads)
+decode_kernel(const Params p) {
+  constexpr int LPK = DH / 8;                    // lanes per key (8 bf16 per lane)
+  constexpr int KPW = 32 / LPK;                  // keys per warp per step
+  constexpr int NG = (kThreads / 32) * KPW;      // key groups per CTA
+  constexpr int UNROLL = 4;
+
+  __shared__ float s_self_k[DH], s_self_v[DH];
+  __shared__ float s_m[NG], s_l[NG];
+  __shared__ float s_acc[NG][DH];
+  __shared__ int s_last;
+
+  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int t = p.len[b];
+  const bool dense = is_dense(p.dense_bits, h);
+  const int Dd = dense ? 1 : p.D;
+  bool active = true;
+  int n_slots = 0, w_lo = 0, n_win = 0, n_keys = 0, n_used = 1;
+  if (t >= p.T_max) {
+    active = false;
+    if (split == 0 && h == 0 && tid == 0) raise_error(RATP_ERR_CAPACITY);
+  } else {
+    n_slots = t / Dd;
+    if (p.W > 0 && !dense) {
+      w_lo = max(0, t - p.W + 1);
+      n_win = t - w_lo;
+    }
+    n_keys = n_slots + n_win;
+    n_used = max(1, (n_keys + p.split_keys - 1) / p.split_keys);
+    if (split >= n_used) active = false;
+  }
+
+  if (active) {
+    const long long bh = (long long)b * p.H + h;
+    const __nv_bfloat16* qrow = p.q + bh * DH;
+    const long long cache_row0 = (long long)b * p.rows_per_b + head_offset(p.dense_bits, h, p.T_max, p.D);
+
+    // ---- split 0: recurrence step, append, ring write, self key ----
+    if (split == 0) {
+      for (int c = tid; c < 2 * DH; c += kThreads) {
+        const int s = c / DH, ch = c % DH;
+        float* st = p.state + ((long long)s * p.B * p.H + bh) * DH + ch;
+        const float x = __bfloat162float((s == 0 ? p.xk : p.xv)[bh * DH + ch]);
+        const float gg = __bfloat162float(p.g[bh * DH + ch]);
+        const float hn = fmaf(gg, *st - x, x);
+        *st = hn;
+        const __nv_bfloat16 hb = __float2bfloat16_rn(hn);
+        (s == 0 ? s_self_k : s_self_v)[ch] = __bfloat162float(hb);
+        if (t % Dd == Dd - 1 && n_slots < p.T_max / Dd)
+          (s == 0 ? p.Kc : p.Vc)[(cache_row0 + n_slots) * DH + ch] = hb;
+        if (p.W > 0)
+          (s == 0 ? p.Kw : p.Vw)[(bh * p.W + t % p.W) * DH + ch] = hb;
+      }
+      if (t % Dd == Dd - 1 && n_slots >= p.T_max / Dd && tid == 0) raise_error(RATP_ERR_CAPACITY);
+      __syncthreads();
+    }
+
+    // ---- stream this split's keys ----
+    const int warp = tid >> 5, lane = tid & 31;
+    const int sub = lane / LPK, li = lane % LPK;
+    const int grp = warp * KPW + sub;
+    const unsigned int sub_mask = (LPK == 32) ? 0xffffffffu : (((1u << LPK) - 1u) << (sub * LPK));
+    float qf[8];
+    {
+      const uint4 qv = *reinterpret_cast<const uint4*>(qrow + li * 8);
+      Elem<__nv_bfloat16>::unpack(qv, qf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) qf[i] *= p.scale_log2;
+    }
+    float m = -INFINITY, l = 0.f, acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+
+    const int k_begin = split * p.split_keys;
+    const int k_end = min(n_keys, k_begin + p.split_keys);
+    for (int k0 = k_begin + grp; k0 < k_end; k0 += NG * UNROLL) {
+      uint4 kv[UNROLL], vv[UNROLL];
+      bool use[UNROLL];
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        const int k = k0 + u * NG;
+        use[u] = false;
+        if (k < k_end) {
+          const __nv_bfloat16 *kr, *vr;
+          if (k < n_slots) {
+            kr = p.Kc + (cache_row0 + k) * DH;
+            vr = p.Vc + (cache_row0 + k) * DH;
+            use[u] = true;
+          } else {
+            const int pos = w_lo + (k - n_slots);
+            const long long rr = (bh * p.W + pos % p.W) * DH;
+            kr = p.Kw + rr;
+            vr = p.Vw + rr;
+            use[u] = (pos % Dd) != (Dd - 1);
+          }
+          if (use[u]) {
+            kv[u] = __ldcs(reinterpret_cast<const uint4*>(kr + li * 8));
+            vv[u] = __ldcs(reinterpret_cast<const uint4*>(vr + li * 8));
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < UNROLL; ++u) {
+        float kf[8];
+        Elem<__nv_bfloat16>::unpack(kv[u], kf);
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s = fmaf(qf[i], kf[i], s);
+#pragma unroll
+        for (int off = LPK / 2; off > 0; off >>= 1) s += __shfl_xor_sync(sub_mask, s, off, LPK);
+        if (use[u]) {
+          float vf[8];
+          Elem<__nv_bfloat16>::unpack(vv[u], vf);
+          const float m_new = fmaxf(m, s);
+          const float alpha = exp2f(m - m_new);
+          const float pj = exp2f(s - m_new);
+          l = l * alpha + pj;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[i] = fmaf(acc[i], alpha, pj * vf[i]);
+          m = m_new;
+        }
+      }
+    }
+    // the query's own key, once, in group 0 of split 0
+    if (split == 0 && grp == 0) {
+      float s = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s = fmaf(qf[i], s_self_k[li * 8 + i], s);
+#pragma unroll
+      for (int off = LPK / 2; off > 0; off >>= 1) s += __shfl_xor_sync(sub_mask, s, off, LPK);
+      const float m_new = fmaxf(m, s);
+      const float alpha = exp2f(m - m_new);
+      const float pj = exp2f(s - m_new);
+      l = l * alpha + pj;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = fmaf(acc[i], alpha, pj * s_self_v[li * 8 + i]);
+      m = m_new;
+    }
+    // ---- merge the key groups of this CTA ----
+    if (li == 0) { s_m[grp] = m; s_l[grp] = l; }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) s_acc[grp][li * 8 + i] = acc[i];
+    __syncthreads();
+    float M = -INFINITY;
+#pragma unroll
+    for (int gi = 0; gi < NG; ++gi) M = fmaxf(M, s_m[gi]);
+    const bool single = (n_used == 1);
+    float* part = p.partial + (bh * p.max_splits + split) * (DH + 2);
+    for (int c = tid; c < DH; c += kThreads) {
+      float L = 0.f, A = 0.f;
+#pragma unroll
+      for (int gi = 0; gi < NG; ++gi) {
+        const float w = (s_m[gi] == -INFINITY) ? 0.f : exp2f(s_m[gi] - M);
+        L = fmaf(s_l[gi], w, L);
+        A = fmaf(s_acc[gi][c], w, A);
+      }
+      if (single) {
+        p.o[bh * DH + c] = __float2bfloat16_rn(A / L);
+      } else {
+        __stcg(part + 2 + c, A);
+        if (c == 0) { __stcg(part, M); __stcg(part + 1, L); }
+      }
+    }
+    if (!single) {
+      __threadfence();
+      __syncthreads();
+      if (tid == 0) {
+        const unsigned int prev = atomicAdd(p.counters + bh, 1u);
+        s_last = (prev == (unsigned int)(n_used - 1));
+      }
+      __syncthreads();
+      if (s_last) {
+        __threadfence();
+        const float* pb = p.partial + bh * p.max_splits * (DH + 2);
+        float MM = -INFINITY;
+        for (int i = 0; i < n_used; ++i) MM = fmaxf(MM, __ldcg(pb + i * (DH + 2)));
+        for (int c = tid; c < DH; c += kThreads) {
+          float L = 0.f, A = 0.f;
+          for (int i = 0; i < n_used; ++i) {
+            const float mi = __ldcg(pb + i * (DH + 2));
+            const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - MM);
+            L = fmaf(__ldcg(pb + i * (DH + 2) + 1), w, L);
+            A = fmaf(__ldcg(pb + i * (DH + 2) + 2 + c), w, A);
+          }
+          p.o[bh * DH + c] = __float2bfloat16_rn(A / L);
+        }
+        if (tid == 0) p.counters[bh] = 0u;
+      }
+    }
+  }
+
+  // ---- the last CTA of the grid advances len ----
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    const unsigned int total = gridDim.x * gridDim.y * gridDim.z;
+    const unsigned int prev = atomicAdd(p.counters + (long long)p.B * p.H, 1u);
+    if (prev == total - 1) {
+      __threadfence();
+      for (int bb = 0; bb < p.B; ++bb) {
+        const int tb = p.len[bb];
+        if (tb < p.T_max) p.len[bb] = tb + 1;
+      }
+      p.counters[(long long)p.B * p.H] = 0u;
+      __threadfence();
+    }
+  }
+}
+
+// ---- prefill -> cache hand-off --------------------------------------------
+struct PackParams {
+  const __nv_bfloat16* hk;
+  const __nv_bfloat16* hv;
+  __nv_bfloat16* Kc;
+  __nv_bfloat16* Vc;
+  __nv_bfloat16* Kw;
+  __nv_bfloat16* Vw;
+  int32_t* len;
+  long long rows_per_b;
+  int B, T, H, D, W, T_max;
+  unsigned long long dense_bits[RATP_MAX_HEADS / 64];
+};
+
+// grid (ceil(rows / rows_per_block), H, B); Dh/8 threads per row, 16 B each.
+template <int DH>
+__global__ void __launch_bounds__(256)
+pack_kernel(const PackParams p) {
+  constexpr int TPR = DH / 8;
+  constexpr int RPB = 256 / TPR;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int r = blockIdx.x * RPB + threadIdx.x / TPR;
+  const int li = threadIdx.x % TPR;
+  const bool dense = is_dense(p.dense_bits, h);
+  const int Dd = dense ? 1 : p.D;
+  const int n_dil = p.T / Dd;
+  const int w_lo = max(0, p.T - p.W);
+  const int n_ring = (p.W > 0) ? (p.T - w_lo) : 0;
+  if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) p.len[b] = p.T;
+  const long long src_base = (long long)b * p.T * p.H * DH + (long long)h * DH + li * 8;
+  if (r < n_dil) {
+    const int pos = r * Dd + Dd - 1;
+    const long long src = src_base + (long long)pos * p.H * DH;
+    const long long dst = ((long long)b * p.rows_per_b + head_offset(p.dense_bits, h, p.T_max, p.D) + r) * DH + li * 8;
+    *reinterpret_cast<uint4*>(p.Kc + dst) = *reinterpret_cast<const uint4*>(p.hk + src);
+    *reinterpret_cast<uint4*>(p.Vc + dst) = *reinterpret_cast<const uint4*>(p.hv + src);
+  } else if (r < n_dil + n_ring) {
+    const int pos = w_lo + (r - n_dil);
+    const long long src = src_base + (long long)pos * p.H * DH;
+    const long long dst = (((long long)b * p.H + h) * p.W + pos % p.W) * DH + li * 8;
+    *reinterpret_cast<uint4*>(p.Kw + dst) = *reinterpret_cast<const uint4*>(p.hk + src);
+    *reinterpret_cast<uint4*>(p.Vw + dst) = *reinterpret_cast<const uint4*>(p.hv + src);
+  }
+}
+
+}  // namespace decode
+}  // namespace ratp

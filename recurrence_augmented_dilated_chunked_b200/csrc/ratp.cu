@@ -1,0 +1,483 @@
+// ratp.cu -- C ABI of the RAT+ sequence-mixer library (one translation unit).
+//
+// Host-side argument checks, workspace/cache carving, TMA tensor-map encoding
+// and kernel launches.  The kernels live in the included headers:
+//   scan.cuh       single-pass chunked scan of the forget-gate recurrence
+//   attn_tc.cuh    tensor-core (TMA + tcgen05) dilated/windowed attention
+//   attn_simt.cuh  CUDA-core attention for fp32 / head dim 64
+//   decode.cuh     cache pack and the fused decode step
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "ratp.h"
+#include "common.cuh"
+#include "scan.cuh"
+#include "sm100.cuh"
+#include "attn_tc.cuh"
+#include "attn_simt.cuh"
+#include "decode.cuh"
+
+using namespace ratp;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? RATP_OK : RATP_ERR_CUDA; }
+
+inline int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? RATP_OK : RATP_ERR_CUDA;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n;
+}
+
+// ---- scan -------------------------------------------------------------------
+struct ScanGeom {
+  int slabs, n_chains, n_chunks_t;
+  long long n_chunks;
+};
+
+int scan_geom(int B, int T, int H, int Dh, int dtype, ScanGeom* g) {
+  if (B < 0 || T < 0 || H < 0 || Dh < 0) return RATP_ERR_ARG;
+  if (dtype != RATP_F32 && dtype != RATP_BF16) return RATP_ERR_ARG;
+  const long long C = (long long)H * Dh;
+  if (C % scan::kSlab != 0 || C > (1ll << 30)) return RATP_ERR_SHAPE;
+  const int chunk = (dtype == RATP_BF16) ? scan::Shape<__nv_bfloat16>::kChunk
+                                         : scan::Shape<float>::kChunk;
+  g->slabs = (int)(C / scan::kSlab);
+  g->n_chains = B * g->slabs;
+  g->n_chunks_t = (T + chunk - 1) / chunk;
+  g->n_chunks = (long long)g->n_chains * g->n_chunks_t;
+  if (g->n_chunks > 0x7fffffffll) return RATP_ERR_SHAPE;
+  return RATP_OK;
+}
+
+template <typename T, int NS>
+int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
+                int B, int Tn, int H, int Dh, const ScanGeom& geo,
+                void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (geo.n_chunks == 0) return RATP_OK;
+  if (ws == nullptr || !aligned16(ws)) return ws == nullptr ? RATP_ERR_ARG : RATP_ERR_ALIGN;
+  if (ws_bytes < scan::workspace_bytes(geo.n_chunks, NS)) return RATP_ERR_CAPACITY;
+  scan::Params<T, NS> p;
+  for (int s = 0; s < NS; ++s) {
+    p.x[s] = static_cast<const T*>(x[s]);
+    p.h[s] = static_cast<T*>(h[s]);
+  }
+  p.g = static_cast<const T*>(g);
+  p.final_state = fs;
+  p.ws = scan::carve(ws, geo.n_chunks, NS);
+  p.B = B; p.Tn = Tn; p.C = H * Dh;
+  p.slabs = geo.slabs; p.n_chains = geo.n_chains; p.n_chunks_t = geo.n_chunks_t;
+  cudaError_t e = cudaMemsetAsync(ws, 0, scan::reset_bytes(geo.n_chunks), st);
+  if (e != cudaSuccess) return RATP_ERR_CUDA;
+  scan::scan_kernel<T, NS><<<(unsigned)geo.n_chunks, scan::kThreads, 0, st>>>(p);
+  return launch_status();
+}
+
+int scan_common(int NS, const void* const* x, const void* g, void* const* h, float* fs,
+                int B, int T, int H, int Dh, int dtype, void* ws, size_t ws_bytes, void* stream) {
+  ScanGeom geo;
+  int rc = scan_geom(B, T, H, Dh, dtype, &geo);
+  if (rc) return rc;
+  if (geo.n_chunks == 0) return RATP_OK;
+  if (g == nullptr) return RATP_ERR_ARG;
+  for (int s = 0; s < NS; ++s) {
+    if (x[s] == nullptr || h[s] == nullptr) return RATP_ERR_ARG;
+    if (!aligned16(x[s]) || !aligned16(h[s])) return RATP_ERR_ALIGN;
+  }
+  if (!aligned16(g)) return RATP_ERR_ALIGN;
+  if (fs != nullptr && !aligned16(fs)) return RATP_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == RATP_BF16) {
+    return NS == 1 ? launch_scan<__nv_bfloat16, 1>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st)
+                   : launch_scan<__nv_bfloat16, 2>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st);
+  }
+  return NS == 1 ? launch_scan<float, 1>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st)
+                 : launch_scan<float, 2>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st);
+}
+
+// ---- head masks -------------------------------------------------------------
+int read_mask(const uint8_t* head_mask, int H, unsigned long long* bits, uint8_t* dense_list,
+              int* n_dense, uint8_t* dil_list, int* n_dil) {
+  if (H > RATP_MAX_HEADS) return RATP_ERR_SHAPE;
+  for (int w = 0; w < RATP_MAX_HEADS / 64; ++w) bits[w] = 0ull;
+  int nd = 0, nl = 0;
+  for (int h = 0; h < H; ++h) {
+    const bool dense = head_mask != nullptr && head_mask[h] != 0;
+    if (dense) {
+      bits[h >> 6] |= 1ull << (h & 63);
+      if (dense_list) dense_list[nd] = (uint8_t)h;
+      ++nd;
+    } else {
+      if (dil_list) dil_list[nl] = (uint8_t)h;
+      ++nl;
+    }
+  }
+  if (n_dense) *n_dense = nd;
+  if (n_dil) *n_dil = nl;
+  return RATP_OK;
+}
+
+int check_attn_args(const void* q, const void* hk, const void* hv, void* o,
+                    int B, int T, int H, int Dh, int D, int W, int dtype) {
+  if (B < 0 || T < 0 || H < 0 || D < 1 || W < 0) return RATP_ERR_ARG;
+  if (dtype != RATP_F32 && dtype != RATP_BF16) return RATP_ERR_ARG;
+  if (Dh != 64 && Dh != 128) return RATP_ERR_SHAPE;
+  if (H > RATP_MAX_HEADS) return RATP_ERR_SHAPE;
+  if ((long long)B * T * H == 0) return RATP_OK;
+  if (!q || !hk || !hv || !o) return RATP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(hk) || !aligned16(hv) || !aligned16(o)) return RATP_ERR_ALIGN;
+  if ((long long)B * T * H * Dh > (1ll << 40)) return RATP_ERR_SHAPE;
+  return RATP_OK;
+}
+
+int launch_attn_simt(const void* q, const void* hk, const void* hv, void* o,
+                     int B, int T, int H, int Dh, int D, int W,
+                     const uint8_t* head_mask, int dtype, cudaStream_t st) {
+  attn_simt::Params p;
+  p.q = q; p.hk = hk; p.hv = hv; p.o = o;
+  p.B = B; p.T = T; p.H = H; p.D = D; p.W = W;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)Dh);
+  int rc = read_mask(head_mask, H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
+  if (rc) return rc;
+  const long long rows = (long long)B * T * H;
+  const unsigned grid = (unsigned)((rows + attn_simt::kWarps - 1) / attn_simt::kWarps);
+  const int threads = attn_simt::kWarps * 32;
+  if (dtype == RATP_BF16) {
+    if (Dh == 128) attn_simt::attn_simt_kernel<__nv_bfloat16, 128><<<grid, threads, 0, st>>>(p);
+    else attn_simt::attn_simt_kernel<__nv_bfloat16, 64><<<grid, threads, 0, st>>>(p);
+  } else {
+    if (Dh == 128) attn_simt::attn_simt_kernel<float, 128><<<grid, threads, 0, st>>>(p);
+    else attn_simt::attn_simt_kernel<float, 64><<<grid, threads, 0, st>>>(p);
+  }
+  return launch_status();
+}
+
+// ---- TMA tensor maps (driver entry point fetched through the runtime) --------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// [B][rows][H][128] bf16 view, rows of `row_stride_elems` elements apart,
+// starting `base_elems` elements into each batch item; box 64 x 1 x 128 x 1.
+bool make_map(CUtensorMap* m, const void* base, long long base_elems, int B, long long rows,
+              int H, long long row_stride_elems, long long batch_stride_elems) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {128 * 2, (cuuint64_t)row_stride_elems * 2,
+                                 (cuuint64_t)batch_stride_elems * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  void* addr = const_cast<char*>(static_cast<const char*>(base)) + base_elems * 2;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, addr, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
+                   int B, int T, int H, int D, int W, const uint8_t* head_mask,
+                   cudaStream_t st) {
+  attn_tc::Params p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.B = B; p.T = T; p.H = H; p.D = D; p.W_eff = W > 0 ? W : 1;
+  p.NQ = (T + attn_tc::BM - 1) / attn_tc::BM;
+  unsigned long long bits[RATP_MAX_HEADS / 64];
+  int rc = read_mask(head_mask, H, bits, p.dense_list, &p.n_dense, p.dil_list, &p.n_dil);
+  if (rc) return rc;
+  p.n_items_dense = B * p.n_dense * p.NQ;
+  p.n_items = B * H * p.NQ;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
+  const long long row = (long long)H * 128, bat = (long long)T * row;
+  CUtensorMap tq, tkp, tvp, tkd, tvd;
+  if (!make_map(&tq, q, 0, B, T, H, row, bat) || !make_map(&tkp, hk, 0, B, T, H, row, bat) ||
+      !make_map(&tvp, hv, 0, B, T, H, row, bat))
+    return RATP_ERR_CUDA;
+  const long long n_slots = T / D;
+  if (n_slots >= 1) {
+    if (!make_map(&tkd, hk, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat) ||
+        !make_map(&tvd, hv, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat))
+      return RATP_ERR_CUDA;
+  } else {
+    tkd = tkp;   // no dilated slot exists for any query: never read
+    tvd = tvp;
+  }
+  static std::once_flag attr_once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(attr_once, [] {
+    attr_err = cudaFuncSetAttribute(attn_tc::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)attn_tc::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return RATP_ERR_CUDA;
+  const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
+  attn_tc::attn_kernel<<<grid, attn_tc::kThreads, attn_tc::kSmemBytes, st>>>(tq, tkp, tvp, tkd, tvd, p);
+  return launch_status();
+}
+
+// ---- cache ------------------------------------------------------------------
+struct CacheLayout {
+  long long rows_per_b;
+  size_t off_kc, off_vc, off_kw, off_vw, off_len, off_part, off_cnt, total;
+  int max_splits, split_keys;
+};
+
+constexpr int kDefaultSplitKeys = 256;
+
+int cache_layout(int B, int H, int Dh, int T_max, int D, int W, const uint8_t* head_mask,
+                 CacheLayout* L) {
+  if (B < 1 || H < 1 || T_max < 1 || D < 1 || W < 0) return RATP_ERR_ARG;
+  if (Dh != 128 && Dh != 64) return RATP_ERR_SHAPE;
+  if (H > RATP_MAX_HEADS) return RATP_ERR_SHAPE;
+  long long per_b = 0;
+  int max_keys = 0;
+  for (int h = 0; h < H; ++h) {
+    const bool dense = head_mask != nullptr && head_mask[h] != 0;
+    const int cap = dense ? T_max : T_max / D;
+    per_b += cap;
+    const int keys = cap + (dense ? 0 : W);
+    if (keys > max_keys) max_keys = keys;
+  }
+  L->rows_per_b = per_b;
+  L->split_keys = kDefaultSplitKeys;
+  L->max_splits = (max_keys + L->split_keys - 1) / L->split_keys;
+  if (L->max_splits < 1) L->max_splits = 1;
+  const size_t row_bytes = (size_t)Dh * 2;
+  size_t off = 0;
+  auto take = [&](size_t bytes) { size_t o = off; off += scan::align256(bytes); return o; };
+  L->off_kc = take((size_t)B * per_b * row_bytes);
+  L->off_vc = take((size_t)B * per_b * row_bytes);
+  L->off_kw = take((size_t)B * H * W * row_bytes);
+  L->off_vw = take((size_t)B * H * W * row_bytes);
+  L->off_len = take((size_t)B * 4);
+  L->off_part = take((size_t)B * H * L->max_splits * (Dh + 2) * 4);
+  L->off_cnt = take((size_t)(B * H + 1) * 4);
+  L->total = off;
+  return RATP_OK;
+}
+
+bool cache_matches(const ratp_cache* c, int D, int W, const uint8_t* head_mask) {
+  if (c->D != D || c->W != W) return false;
+  for (int h = 0; h < c->H; ++h) {
+    const uint8_t want = (head_mask != nullptr && head_mask[h] != 0) ? 1 : 0;
+    if (c->dense[h] != want) return false;
+  }
+  return true;
+}
+
+}  // namespace
+
+// =============================================================================
+extern "C" {
+
+const char* ratp_status_string(int status) {
+  switch (status) {
+    case RATP_OK: return "ok";
+    case RATP_ERR_ARG: return "invalid argument";
+    case RATP_ERR_SHAPE: return "unsupported shape";
+    case RATP_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case RATP_ERR_CAPACITY: return "workspace or cache capacity exceeded";
+    case RATP_ERR_TIMEOUT: return "bounded device wait expired";
+    case RATP_ERR_CUDA: return "CUDA error";
+    case RATP_ERR_UNSUPPORTED: return "unsupported dtype/shape combination";
+    default: return "unknown status";
+  }
+}
+
+int ratp_last_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return RATP_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, ratp::g_error_word, sizeof(word)) != cudaSuccess) return RATP_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(ratp::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return RATP_ERR_CUDA;
+  for (int code = 1; code < 32; ++code)
+    if (word & (1u << code)) return code;
+  return RATP_OK;
+}
+
+int ratp_device_sm_count(int* sms) {
+  if (!sms) return RATP_ERR_ARG;
+  *sms = sm_count();
+  return RATP_OK;
+}
+
+int ratp_scan_workspace_bytes(int B, int T, int H, int Dh, int dtype, size_t* bytes) {
+  if (!bytes) return RATP_ERR_ARG;
+  ScanGeom geo;
+  int rc = scan_geom(B, T, H, Dh, dtype, &geo);
+  if (rc) return rc;
+  // one size serves both the single- and the two-stream scan
+  *bytes = scan::workspace_bytes(geo.n_chunks, 2);
+  return RATP_OK;
+}
+
+int ratp_scan_prefill(const void* x, const void* g, void* h, float* final_state,
+                      int B, int T, int H, int Dh, int dtype,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  const void* xs[1] = {x};
+  void* hs[1] = {h};
+  return scan_common(1, xs, g, hs, final_state, B, T, H, Dh, dtype, workspace, workspace_bytes, stream);
+}
+
+int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
+                         void* hk, void* hv, float* final_state,
+                         int B, int T, int H, int Dh, int dtype,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  const void* xs[2] = {xk, xv};
+  void* hs[2] = {hk, hv};
+  return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, workspace, workspace_bytes, stream);
+}
+
+int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv, void* o,
+                                   int B, int T, int H, int Dh, int D, int W,
+                                   const uint8_t* head_mask, int dtype, void* stream) {
+  int rc = check_attn_args(q, hk, hv, o, B, T, H, Dh, D, W, dtype);
+  if (rc) return rc;
+  if ((long long)B * T * H == 0) return RATP_OK;
+  return launch_attn_simt(q, hk, hv, o, B, T, H, Dh, D, W, head_mask, dtype,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int ratp_dilated_attn_prefill(const void* q, const void* hk, const void* hv, void* o,
+                              int B, int T, int H, int Dh, int D, int W,
+                              const uint8_t* head_mask, int dtype, void* stream) {
+  int rc = check_attn_args(q, hk, hv, o, B, T, H, Dh, D, W, dtype);
+  if (rc) return rc;
+  if ((long long)B * T * H == 0) return RATP_OK;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == RATP_BF16 && Dh == 128)
+    return launch_attn_tc(q, hk, hv, o, B, T, H, D, W, head_mask, st);
+  return launch_attn_simt(q, hk, hv, o, B, T, H, Dh, D, W, head_mask, dtype, st);
+}
+
+int ratp_cache_bytes(int B, int H, int Dh, int T_max, int D, int W,
+                     const uint8_t* head_mask, size_t* bytes) {
+  if (!bytes) return RATP_ERR_ARG;
+  CacheLayout L;
+  int rc = cache_layout(B, H, Dh, T_max, D, W, head_mask, &L);
+  if (rc) return rc;
+  *bytes = L.total;
+  return RATP_OK;
+}
+
+int ratp_cache_init(ratp_cache* c, void* buffer, size_t bytes, int B, int H, int Dh, int T_max,
+                    int D, int W, const uint8_t* head_mask, void* stream) {
+  if (!c || !buffer) return RATP_ERR_ARG;
+  if (!aligned16(buffer)) return RATP_ERR_ALIGN;
+  CacheLayout L;
+  int rc = cache_layout(B, H, Dh, T_max, D, W, head_mask, &L);
+  if (rc) return rc;
+  if (bytes < L.total) return RATP_ERR_CAPACITY;
+  char* base = static_cast<char*>(buffer);
+  memset(c, 0, sizeof(*c));
+  c->Kc = base + L.off_kc;
+  c->Vc = base + L.off_vc;
+  c->Kw = W > 0 ? base + L.off_kw : nullptr;
+  c->Vw = W > 0 ? base + L.off_vw : nullptr;
+  c->len = reinterpret_cast<int32_t*>(base + L.off_len);
+  c->partial = reinterpret_cast<float*>(base + L.off_part);
+  c->counters = reinterpret_cast<uint32_t*>(base + L.off_cnt);
+  c->rows_per_b = L.rows_per_b;
+  c->B = B; c->H = H; c->Dh = Dh; c->T_max = T_max; c->D = D; c->W = W;
+  c->split_keys = L.split_keys;
+  c->max_splits = L.max_splits;
+  for (int h = 0; h < H; ++h) c->dense[h] = (head_mask != nullptr && head_mask[h] != 0) ? 1 : 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(c->len, 0, (size_t)B * 4, st) != cudaSuccess) return RATP_ERR_CUDA;
+  if (cudaMemsetAsync(c->counters, 0, (size_t)(B * H + 1) * 4, st) != cudaSuccess) return RATP_ERR_CUDA;
+  return RATP_OK;
+}
+
+int ratp_cache_pack(ratp_cache* c, const void* hk, const void* hv, int T, void* stream) {
+  if (!c || !hk || !hv) return RATP_ERR_ARG;
+  if (T < 0 || T > c->T_max) return RATP_ERR_CAPACITY;
+  if (!aligned16(hk) || !aligned16(hv)) return RATP_ERR_ALIGN;
+  decode::PackParams p;
+  p.hk = static_cast<const __nv_bfloat16*>(hk);
+  p.hv = static_cast<const __nv_bfloat16*>(hv);
+  p.Kc = static_cast<__nv_bfloat16*>(c->Kc);
+  p.Vc = static_cast<__nv_bfloat16*>(c->Vc);
+  p.Kw = static_cast<__nv_bfloat16*>(c->Kw);
+  p.Vw = static_cast<__nv_bfloat16*>(c->Vw);
+  p.len = c->len;
+  p.rows_per_b = c->rows_per_b;
+  p.B = c->B; p.T = T; p.H = c->H; p.D = c->D; p.W = c->W; p.T_max = c->T_max;
+  int rc = read_mask(c->dense, c->H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
+  if (rc) return rc;
+  int max_rows = 0;
+  for (int h = 0; h < c->H; ++h) {
+    const int Dd = c->dense[h] ? 1 : c->D;
+    const int rows = T / Dd + (c->W > 0 ? (T < c->W ? T : c->W) : 0);
+    if (rows > max_rows) max_rows = rows;
+  }
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int rpb = 256 / (c->Dh / 8);
+  dim3 grid((unsigned)((max_rows + rpb - 1) / rpb), (unsigned)c->H, (unsigned)c->B);
+  if (grid.x == 0) grid.x = 1;   // still sets len
+  if (c->Dh == 128) decode::pack_kernel<128><<<grid, 256, 0, st>>>(p);
+  else decode::pack_kernel<64><<<grid, 256, 0, st>>>(p);
+  return launch_status();
+}
+
+int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* g,
+                     float* state, ratp_cache* c, void* o,
+                     int D, int W, const uint8_t* head_mask, void* stream) {
+  if (!q || !xk || !xv || !g || !state || !c || !o) return RATP_ERR_ARG;
+  if (!aligned16(q) || !aligned16(xk) || !aligned16(xv) || !aligned16(g) || !aligned16(state) ||
+      !aligned16(o))
+    return RATP_ERR_ALIGN;
+  if (!cache_matches(c, D, W, head_mask)) return RATP_ERR_ARG;
+  decode::Params p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.xk = static_cast<const __nv_bfloat16*>(xk);
+  p.xv = static_cast<const __nv_bfloat16*>(xv);
+  p.g = static_cast<const __nv_bfloat16*>(g);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.state = state;
+  p.Kc = static_cast<__nv_bfloat16*>(c->Kc);
+  p.Vc = static_cast<__nv_bfloat16*>(c->Vc);
+  p.Kw = static_cast<__nv_bfloat16*>(c->Kw);
+  p.Vw = static_cast<__nv_bfloat16*>(c->Vw);
+  p.len = c->len;
+  p.partial = c->partial;
+  p.counters = c->counters;
+  p.rows_per_b = c->rows_per_b;
+  p.B = c->B; p.H = c->H; p.D = c->D; p.W = c->W; p.T_max = c->T_max;
+  p.split_keys = c->split_keys;
+  p.max_splits = c->max_splits;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)c->Dh);
+  int rc = read_mask(c->dense, c->H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  dim3 grid((unsigned)c->max_splits, (unsigned)c->H, (unsigned)c->B);
+  if (c->Dh == 128) decode::decode_kernel<128><<<grid, decode::kThreads, 0, st>>>(p);
+  else decode::decode_kernel<64><<<grid, decode::kThreads, 0, st>>>(p);
+  return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,127 @@
+"""CPU checks of the C ABI: the library builds, loads, exports every function
+that ``include/ratp.h`` declares, and rejects bad arguments on the host before
+touching the GPU (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+import recurrence_augmented_dilated_chunked_b200 as ratp
+from recurrence_augmented_dilated_chunked_b200 import _binding, build
+
+HEADER = os.path.join(ROOT, "include", "ratp.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:int|const char\*)\s+(ratp_\w+)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_library()
+    return ratp.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert len(declared) >= 12
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert set(declared) == set(_binding.exported_symbols())
+
+
+def _struct_fields(body):
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    names = []
+    for decl in body.split(";"):
+        parts = [x.strip() for x in decl.strip().split(",") if x.strip()]
+        if not parts:
+            continue
+        names.append(parts[0].split()[-1].lstrip("*"))
+        names.extend(x.lstrip("*") for x in parts[1:])
+    return [re.sub(r"\[.*\]", "", n) for n in names]
+
+
+def test_cache_struct_matches_header():
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct ratp_cache \{(.*?)\} ratp_cache;", src, re.S).group(1)
+    assert _struct_fields(body) == [f[0] for f in _binding.CacheStruct._fields_]
+
+
+def test_status_strings(lib):
+    assert lib.ratp_status_string(0) == b"ok"
+    assert b"aligned" in lib.ratp_status_string(3)
+
+
+def test_scan_workspace_query(lib):
+    n = ctypes.c_size_t()
+    assert lib.ratp_scan_workspace_bytes(8, 4096, 16, 128, 1, ctypes.byref(n)) == 0
+    chunks = 8 * (2048 // 64) * (4096 // 128)
+    assert n.value >= chunks * (4 + 4 * 64 * 5)
+    assert lib.ratp_scan_workspace_bytes(1, 10, 1, 32, 1, ctypes.byref(n)) == 2   # H*Dh % 64
+    assert lib.ratp_scan_workspace_bytes(-1, 10, 1, 64, 1, ctypes.byref(n)) == 1
+    assert lib.ratp_scan_workspace_bytes(1, 10, 1, 64, 7, ctypes.byref(n)) == 1
+
+
+def test_cache_bytes_query(lib):
+    n = ctypes.c_size_t()
+    assert lib.ratp_cache_bytes(64, 16, 128, 33024, 64, 128, None, ctypes.byref(n)) == 0
+    rows = 64 * 16 * (33024 // 64)
+    ring = 64 * 16 * 128
+    assert n.value >= 2 * (rows + ring) * 256
+    mask = (ctypes.c_uint8 * 4)(1, 0, 0, 0)
+    m = ctypes.c_size_t()
+    assert lib.ratp_cache_bytes(1, 4, 128, 64, 4, 0, ctypes.cast(mask, ctypes.c_void_p), ctypes.byref(m)) == 0
+    assert m.value >= 2 * (64 + 3 * 16) * 256
+    assert lib.ratp_cache_bytes(1, 4, 96, 64, 4, 0, None, ctypes.byref(m)) == 2
+    assert lib.ratp_cache_bytes(1, 4, 128, 64, 0, 0, None, ctypes.byref(m)) == 1
+
+
+def test_attention_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)
+    # D < 1, W < 0, Dh unsupported, null pointers, misaligned pointers
+    assert lib.ratp_dilated_attn_prefill(p, p, p, p, 1, 8, 1, 128, 0, 0, None, 1, None) == 1
+    assert lib.ratp_dilated_attn_prefill(p, p, p, p, 1, 8, 1, 128, 2, -1, None, 1, None) == 1
+    assert lib.ratp_dilated_attn_prefill(p, p, p, p, 1, 8, 1, 96, 2, 0, None, 1, None) == 2
+    assert lib.ratp_dilated_attn_prefill(None, p, p, p, 1, 8, 1, 128, 2, 0, None, 1, None) == 1
+    q = ctypes.c_void_p(24)
+    assert lib.ratp_dilated_attn_prefill(q, p, p, p, 1, 8, 1, 128, 2, 0, None, 1, None) == 3
+    assert lib.ratp_dilated_attn_prefill_simt(p, p, p, p, 1, 8, 300, 64, 2, 0, None, 0, None) == 2
+    # empty problem: nothing to do, no launch
+    assert lib.ratp_dilated_attn_prefill(None, None, None, None, 0, 8, 1, 128, 2, 0, None, 1, None) == 0
+
+
+def test_scan_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.ratp_scan_prefill(None, p, p, None, 1, 8, 1, 64, 1, p, 1 << 20, None) == 1
+    assert lib.ratp_scan_prefill(ctypes.c_void_p(8), p, p, None, 1, 8, 1, 64, 1, p, 1 << 20, None) == 3
+    # workspace too small
+    assert lib.ratp_scan_prefill(p, p, p, None, 1, 8, 1, 64, 1, p, 16, None) == 4
+    assert lib.ratp_scan_prefill_kv(p, p, p, p, p, None, 1, 8, 1, 64, 1, None, 1 << 20, None) == 1
+    # T == 0 is a no-op
+    assert lib.ratp_scan_prefill(None, None, None, None, 1, 0, 1, 64, 1, None, 0, None) == 0
+
+
+def test_decode_rejects_mismatched_cache_on_host(lib):
+    c = _binding.CacheStruct()
+    c.D, c.W, c.H = 4, 0, 2
+    p = ctypes.c_void_p(16)
+    assert lib.ratp_decode_step(p, p, p, p, p, ctypes.byref(c), p, 8, 0, None, None) == 1
+    assert lib.ratp_decode_step(p, p, p, p, p, ctypes.byref(c), p, 4, 3, None, None) == 1
+    mask = (ctypes.c_uint8 * 2)(1, 0)
+    assert lib.ratp_decode_step(p, p, p, p, p, ctypes.byref(c), p, 4, 0,
+                                ctypes.cast(mask, ctypes.c_void_p), None) == 1
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    saved = _binding._lib
+    _binding._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="missing"):
+            _binding.load_library(str(tmp_path / "nope.so"))
+    finally:
+        _binding._lib = saved
