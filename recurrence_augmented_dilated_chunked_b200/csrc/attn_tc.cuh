@@ -272,7 +272,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       float m_used = -1e30f, l = 0.f;
       for (int j = 0; j < it.n_tiles; ++j, ++g) {
         const int sbuf = g & 1;
-        if (!mbar_wait(b_sfull + 8 * sbuf, (g >> 1) & 1, s_abort)) { ok = false; break; }
+        if (!warp_all(mbar_wait(b_sfull + 8 * sbuf, (g >> 1) & 1, s_abort))) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[BN];
 #pragma unroll
@@ -304,12 +304,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           }
         }
         // previous P.V must be complete before P is overwritten / O rescaled
-        if (g > 0 && !mbar_wait(b_pvdone, (g - 1) & 1, s_abort)) { ok = false; break; }
+        if (g > 0 && !warp_all(mbar_wait(b_pvdone, (g - 1) & 1, s_abort))) { ok = false; break; }
         tc_fence_after();
-        if (j == 0) {
-          m_used = fmaxf(mx, -1e30f);
-        } else if (mx > m_used + kRescaleThreshold) {
-          const float alpha = exp2f(m_used - mx);
+        // O is rescaled only when some row's running max grew by more than
+        // 2^kRescaleThreshold.  tcgen05.ld/st are warp-collective, so the
+        // decision is taken per warp and rows that do not need it use alpha 1.
+        const bool need = (j > 0) && (mx > m_used + kRescaleThreshold);
+        if (j == 0) m_used = fmaxf(mx, -1e30f);
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? exp2f(m_used - mx) : 1.f;
 #pragma unroll
           for (int c = 0; c < DH / 32; ++c) {
             uint32_t o32[32];
@@ -320,8 +323,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             tmem_st32(tl + kColO + c * 32, o32);
           }
           tmem_wait_st();
-          l *= alpha;
-          m_used = mx;
+          if (need) {
+            l *= alpha;
+            m_used = mx;
+          }
         }
         float rowsum = 0.f;
 #pragma unroll
@@ -345,7 +350,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> global
-      if (!mbar_wait(b_pvdone, (g - 1) & 1, s_abort)) { ok = false; break; }
+      if (!warp_all(mbar_wait(b_pvdone, (g - 1) & 1, s_abort))) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.f / l;
       __nv_bfloat16* orow = p.o + (((size_t)it.b * p.T + t) * p.H + it.h) * DH;

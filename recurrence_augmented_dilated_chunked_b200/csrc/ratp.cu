@@ -11,6 +11,8 @@
 #include <string.h>
 
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "ratp.h"
 #include "common.cuh"
@@ -26,11 +28,25 @@ namespace {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inline int cuda_status(cudaError_t e) { return e == cudaSuccess ? RATP_OK : RATP_ERR_CUDA; }
-
 inline int launch_status() {
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? RATP_OK : RATP_ERR_CUDA;
+}
+
+// Opt a kernel into more than 48 KB of dynamic shared memory, once per device.
+template <typename F>
+bool ensure_smem(F* func, int bytes) {
+  static std::mutex mu;
+  static std::set<std::pair<const void*, int>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_pair(reinterpret_cast<const void*>(func), dev);
+  if (done.count(key)) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done.insert(key);
+  return true;
 }
 
 int sm_count() {
@@ -61,6 +77,28 @@ int scan_geom(int B, int T, int H, int Dh, int dtype, ScanGeom* g) {
   return RATP_OK;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+
+// [B][T][C] view, box of 64 channels x `rows` tokens x 1 sequence, no swizzle.
+template <typename T>
+bool make_scan_map(CUtensorMap* m, const void* base, int B, int Tn, int C, int rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const CUtensorMapDataType dt = sizeof(T) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)Tn, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)C * sizeof(T), (cuuint64_t)Tn * C * sizeof(T)};
+  const cuuint32_t box[3] = {(cuuint32_t)scan::kSlab, (cuuint32_t)rows, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T, int NS>
 int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
                 int B, int Tn, int H, int Dh, const ScanGeom& geo,
@@ -69,18 +107,25 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   if (ws == nullptr || !aligned16(ws)) return ws == nullptr ? RATP_ERR_ARG : RATP_ERR_ALIGN;
   if (ws_bytes < scan::workspace_bytes(geo.n_chunks, NS)) return RATP_ERR_CAPACITY;
   scan::Params<T, NS> p;
-  for (int s = 0; s < NS; ++s) {
-    p.x[s] = static_cast<const T*>(x[s]);
-    p.h[s] = static_cast<T*>(h[s]);
-  }
-  p.g = static_cast<const T*>(g);
+  for (int s = 0; s < NS; ++s) p.h[s] = static_cast<T*>(h[s]);
   p.final_state = fs;
   p.ws = scan::carve(ws, geo.n_chunks, NS);
   p.B = B; p.Tn = Tn; p.C = H * Dh;
   p.slabs = geo.slabs; p.n_chains = geo.n_chains; p.n_chunks_t = geo.n_chunks_t;
+  const int C = H * Dh, rows = scan::Shape<T>::kChunk;
+  CUtensorMap tg, tx0, tx1;
+  if (!make_scan_map<T>(&tg, g, B, Tn, C, rows) || !make_scan_map<T>(&tx0, x[0], B, Tn, C, rows))
+    return RATP_ERR_CUDA;
+  if (NS == 2) {
+    if (!make_scan_map<T>(&tx1, x[1], B, Tn, C, rows)) return RATP_ERR_CUDA;
+  } else {
+    tx1 = tx0;
+  }
+  constexpr int smem = scan::Smem<T, NS>::kBytes;
+  if (!ensure_smem(scan::scan_kernel<T, NS>, smem)) return RATP_ERR_CUDA;
   cudaError_t e = cudaMemsetAsync(ws, 0, scan::reset_bytes(geo.n_chunks), st);
   if (e != cudaSuccess) return RATP_ERR_CUDA;
-  scan::scan_kernel<T, NS><<<(unsigned)geo.n_chunks, scan::kThreads, 0, st>>>(p);
+  scan::scan_kernel<T, NS><<<(unsigned)geo.n_chunks, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);
   return launch_status();
 }
 
@@ -164,11 +209,6 @@ int launch_attn_simt(const void* q, const void* hk, const void* hv, void* o,
 }
 
 // ---- TMA tensor maps (driver entry point fetched through the runtime) --------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 EncodeTiledFn encode_fn() {
   static EncodeTiledFn fn = nullptr;
   static std::once_flag once;
@@ -227,13 +267,7 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
     tkd = tkp;   // no dilated slot exists for any query: never read
     tvd = tvp;
   }
-  static std::once_flag attr_once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(attr_once, [] {
-    attr_err = cudaFuncSetAttribute(attn_tc::attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)attn_tc::kSmemBytes);
-  });
-  if (attr_err != cudaSuccess) return RATP_ERR_CUDA;
+  if (!ensure_smem(attn_tc::attn_kernel, (int)attn_tc::kSmemBytes)) return RATP_ERR_CUDA;
   const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
   attn_tc::attn_kernel<<<grid, attn_tc::kThreads, attn_tc::kSmemBytes, st>>>(tq, tkp, tvp, tkd, tvd, p);
   return launch_status();
