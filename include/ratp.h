@@ -100,6 +100,35 @@ int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Allocation-free variant of ratp_scan_prefill_kv.  The paper has no
+ * counterpart: this is a convenience of the library.
+ *
+ * It serves callers that must not allocate device memory themselves and so
+ * cannot hand in the scratch workspace that ratp_scan_prefill_kv needs --
+ * for example a plug-in running inside a host application whose memory pool
+ * owns every device byte, or a latency-critical path where cudaMalloc's
+ * implicit device-wide synchronisation is not acceptable.  The scratch is a
+ * fixed array of RATP_NOALLOC_SCRATCH_BYTES (16 MiB) compiled into the
+ * library's device image; every device that loads the library holds it until
+ * the process exits.  Inputs, outputs and errors are those of
+ * ratp_scan_prefill_kv (the caller still provides and owns all tensors), and
+ * the call itself performs no allocation of any kind.
+ *   - A shape whose scratch would not fit returns RATP_ERR_CAPACITY
+ *     (bf16: at most ~13,000 chunks of 128 tokens x 64 channels, i.e.
+ *     B*T*H*Dh up to ~106 million elements; fp32 chunks hold 64 tokens).
+ *   - The first call on a device looks up the array's device address with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls share the one array, which keeps the previous call's
+ *     contents; each call clears, on `stream`, the part that must start at
+ *     zero.  Calls that can run at the same time on the GPU (for example on
+ *     two unordered streams) race on the array and produce wrong results.
+ * ---------------------------------------------------------------------- */
+#define RATP_NOALLOC_SCRATCH_BYTES (16u << 20)
+int ratp_scan_prefill_kv_noalloc(const void* xk, const void* xv, const void* g,
+                                 void* hk, void* hv, float* final_state,
+                                 int B, int T, int H, int Dh, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
  * Dilated (+ windowed) prefill attention (RAT+ abstract; write-up sections 1
  * and 6).
  *

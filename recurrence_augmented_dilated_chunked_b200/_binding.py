@@ -54,6 +54,7 @@ _SIGS = {
     "ratp_scan_workspace_bytes": ([_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "ratp_scan_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "ratp_scan_prefill_kv": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
+    "ratp_scan_prefill_kv_noalloc": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P], _I),
     "ratp_dilated_attn_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_simt": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_cache_bytes": ([_I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)], _I),
@@ -169,6 +170,25 @@ def scan_prefill_kv(xk, xv, g, hk=None, hv=None, final_state=None, workspace=Non
     _check("ratp_scan_prefill_kv", lib.ratp_scan_prefill_kv(
         _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(final_state),
         B, T, H, Dh, _DTYPE[xk.dtype], _ptr(ws), ws.numel(), _stream(xk)))
+    return hk, hv
+
+
+def scan_prefill_kv_noalloc(xk, xv, g, hk, hv, final_state=None):
+    """(hk, hv) like ``scan_prefill_kv``, but the library supplies the scratch
+    from its fixed device array, so nothing is allocated for the call (the
+    outputs hk and hv must be passed in)."""
+    lib = load_library()
+    _need(xk, "xk")
+    _need(xv, "xv", xk.dtype)
+    _need(g, "g", xk.dtype)
+    _need(hk, "hk", xk.dtype)
+    _need(hv, "hv", xk.dtype)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32)
+    B, T, H, Dh = xk.shape
+    _check("ratp_scan_prefill_kv_noalloc", lib.ratp_scan_prefill_kv_noalloc(
+        _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(final_state),
+        B, T, H, Dh, _DTYPE[xk.dtype], _stream(xk)))
     return hk, hv
 
 

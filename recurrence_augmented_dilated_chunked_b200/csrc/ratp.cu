@@ -323,6 +323,28 @@ bool cache_matches(const ratp_cache* c, int D, int W, const uint8_t* head_mask) 
   return true;
 }
 
+// ---- allocation-free scan scratch ---------------------------------------------
+// One fixed array in the device image; its device address is looked up once
+// per device (cudaGetSymbolAddress with that device current) and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RATP_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return RATP_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return RATP_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return RATP_OK;
+}
+
 }  // namespace
 
 // =============================================================================
@@ -385,6 +407,23 @@ int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
   const void* xs[2] = {xk, xv};
   void* hs[2] = {hk, hv};
   return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, workspace, workspace_bytes, stream);
+}
+
+int ratp_scan_prefill_kv_noalloc(const void* xk, const void* xv, const void* g,
+                                 void* hk, void* hv, float* final_state,
+                                 int B, int T, int H, int Dh, int dtype, void* stream) {
+  ScanGeom geo;
+  int rc = scan_geom(B, T, H, Dh, dtype, &geo);
+  if (rc) return rc;
+  if (geo.n_chunks == 0) return RATP_OK;
+  if (scan::workspace_bytes(geo.n_chunks, 2) > (size_t)RATP_NOALLOC_SCRATCH_BYTES) return RATP_ERR_CAPACITY;
+  void* ws = nullptr;
+  rc = noalloc_scratch(&ws);
+  if (rc) return rc;
+  const void* xs[2] = {xk, xv};
+  void* hs[2] = {hk, hv};
+  return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, ws,
+                     (size_t)RATP_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv, void* o,
