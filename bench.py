@@ -84,6 +84,22 @@ def decode_bytes_per_step(w, t):
     return total
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(values, world, device=None):
+    """Element-wise max of per-rank timings (every rank calls it, same order)."""
+    if world == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(units_per_rank, world, seconds_max):
+    """Whole-job throughput of weak-scaled replicas: all ranks' units over the
+    slowest rank's time."""
+    return world * units_per_rank / seconds_max
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi samples during the timed region (clocks and throttle reasons)."""
@@ -326,15 +342,8 @@ def run_ours(args, rank, world, local_rank):
     ratp.last_error(dev)
 
     # ---- max over ranks ----
-    def rmax(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
-
-    s_scan, s_attn, s_dec = rmax(sum(scan_ms)), rmax(sum(attn_ms)), rmax(sum(dec_ms))
-    s_total, s_e2e = rmax(total_ms), rmax(e2e_ms)
+    s_scan, s_attn, s_dec, s_total, s_e2e = max_over_ranks(
+        [sum(scan_ms), sum(attn_ms), sum(dec_ms), total_ms, e2e_ms], world, dev)
     if rank != 0:
         return 0
 
@@ -343,8 +352,8 @@ def run_ours(args, rank, world, local_rank):
     peaks = measured_peaks()
     prefill_tokens = wp.B * wp.T
     prefill_s = (s_scan + s_attn) / 1e3
-    value = world * prefill_tokens * K / prefill_s
-    decode_tok_s = world * wd.B * steps * K / (s_dec / 1e3)
+    value = job_throughput(prefill_tokens * K, world, prefill_s)
+    decode_tok_s = job_throughput(wd.B * steps * K, world, s_dec / 1e3)
     scan_gbs = pc["scan_bytes"] * K / (s_scan / 1e3) / 1e9
     attn_gbs = pc["attn_bytes"] * K / (s_attn / 1e3) / 1e9
     attn_tfs = pc["attn_flops"] * K / (s_attn / 1e3) / 1e12
@@ -383,7 +392,7 @@ def run_ours(args, rank, world, local_rank):
                    "graph": "256 decode launches per CUDA graph"},
         "kernels": kernels,
         "roofline": roof,
-        "e2e": {"value": world * prefill_tokens * args.steps / (s_e2e / 1e3), "unit": "tokens/s",
+        "e2e": {"value": job_throughput(prefill_tokens * args.steps, world, s_e2e / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "prefill through the C ABI from pinned host q/xk/xv/g to host o"},
         "gpu_launches": K * (2 + steps),

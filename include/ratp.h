@@ -114,8 +114,8 @@ int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
  * ratp_scan_prefill_kv (the caller still provides and owns all tensors), and
  * the call itself performs no allocation of any kind.
  *   - A shape whose scratch would not fit returns RATP_ERR_CAPACITY
- *     (bf16: at most ~13,000 chunks of 128 tokens x 64 channels, i.e.
- *     B*T*H*Dh up to ~106 million elements; fp32 chunks hold 64 tokens).
+ *     (bf16: at most ~11,900 chunks of 128 tokens x 64 channels, i.e.
+ *     B*T*H*Dh up to ~97 million elements; fp32 chunks hold 64 tokens).
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *   - All calls share the one array, which keeps the previous call's

@@ -19,14 +19,20 @@
 // Per-row validity is a prefix (dilated: s < floor(t / D_h), dense: s <= t) or
 // a range minus a periodic pattern (window), evaluated in registers.
 //
-// Roles (192 threads, one CTA per SM, persistent over items in heavy-first
+// Roles (352 threads, one CTA per SM, persistent over items in heavy-first
 // order -- dense heads and late query tiles first, round-robin over CTAs):
-//   warps 0-3  softmax: thread r owns query row r = TMEM lane r.  Reads S from
-//              TMEM, masks, keeps the running max (rescaling O in TMEM only
-//              when the max grows by more than 2^8), writes P (bf16) into a
-//              128B-swizzled K-major smem tile, and finally normalises O.
-//   warp 4     TMA producer: Q (double-buffered) and a 2-stage K/V ring.
-//   warp 5     allocates TMEM (512 columns: S ping-pong 2x128, O 128) and one
+//   warps 0-7  softmax: warps w and w+4 share query rows 32(w%4)..+31 (TMEM
+//              lanes) and split the 128 key columns in halves.  Each reads its
+//              half of S from TMEM, masks it per 32-column chunk with a bit
+//              mask (all-valid and all-masked chunks take fast paths), the
+//              pair exchanges the row max through shared memory, the running
+//              max is kept with O rescaled in TMEM only when it grows by more
+//              than 2^8, and P (bf16) is written into one of two 128B-swizzled
+//              K-major smem tiles; finally each thread normalises half an O row.
+//   warp 8     TMA producer of Q and of a 2-stage K ring (a K stage is freed
+//              as soon as its S = Q K^T completes);
+//   warp 10    TMA producer of a 2-stage V ring (freed when P V completes);
+//   warp 9     allocates TMEM (512 columns: S ping-pong 2x128, O 128) and one
 //              lane issues S = Q K^T (SS, K-major) and O += P V (P K-major,
 //              V MN-major) as 128x128x16 tcgen05.mma; completions signal
 //              mbarriers via tcgen05.commit.
@@ -42,16 +48,22 @@ constexpr int BM = 128;          // queries per tile
 constexpr int BN = 128;          // keys per tile
 constexpr int DH = 128;          // head dim
 constexpr int NST = 2;           // K/V pipeline stages
-constexpr int kThreads = 192;
+constexpr int kSoftmaxWarps = 8;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kVProducerWarp = 10;
+constexpr int kThreads = 352;
 constexpr uint32_t kHalf = BN * 64 * 2;        // one 64-column half tile: 16 KB
 constexpr uint32_t kTile = 2 * kHalf;          // 128 x 128 bf16: 32 KB
-constexpr uint32_t kOffQ = 0;                  // 2 Q buffers
-constexpr uint32_t kOffK = kOffQ + 2 * kTile;
+constexpr uint32_t kOffQ = 0;                  // Q
+constexpr uint32_t kOffK = kOffQ + kTile;
 constexpr uint32_t kOffV = kOffK + NST * kTile;
-constexpr uint32_t kOffP = kOffV + NST * kTile;
-constexpr uint32_t kOffBar = kOffP + kTile;
-constexpr uint32_t kNumBars = 14;
-constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + alignment slack
+constexpr uint32_t kOffP = kOffV + NST * kTile;  // 2 P buffers
+constexpr uint32_t kOffBar = kOffP + 2 * kTile;
+constexpr uint32_t kNumBars = 18;
+constexpr uint32_t kOffXchg = kOffBar + kNumBars * 8 + 16;     // row-max / row-sum exchange
+constexpr uint32_t kXchgBytes = 2 * BM * 4;                    // [2 halves][128] f32
+constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S buffers at columns 0 and 128
 constexpr uint32_t kColO = 256;    // O at columns 256..383
@@ -123,41 +135,46 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV, sP = sb + kOffP;
   const uint32_t bar0 = sb + kOffBar;
   // barrier map
-  const uint32_t b_qfull = bar0 + 0 * 8;    // [2]
-  const uint32_t b_qempty = bar0 + 2 * 8;   // [2]
-  const uint32_t b_kvfull = bar0 + 4 * 8;   // [NST]
-  const uint32_t b_kvempty = bar0 + 6 * 8;  // [NST]
-  const uint32_t b_sfull = bar0 + 8 * 8;    // [2]
-  const uint32_t b_sfree = bar0 + 10 * 8;   // [2]
-  const uint32_t b_pfull = bar0 + 12 * 8;
-  const uint32_t b_pvdone = bar0 + 13 * 8;
+  const uint32_t b_qfull = bar0 + 0 * 8;
+  const uint32_t b_qempty = bar0 + 1 * 8;
+  const uint32_t b_kfull = bar0 + 2 * 8;    // [NST]
+  const uint32_t b_kempty = bar0 + 4 * 8;   // [NST]
+  const uint32_t b_sfull = bar0 + 6 * 8;    // [2]
+  const uint32_t b_sfree = bar0 + 8 * 8;    // [2]
+  const uint32_t b_pfull = bar0 + 10 * 8;   // [2]
+  const uint32_t b_pvdone = bar0 + 12 * 8;  // [2]
+  const uint32_t b_vfull = bar0 + 14 * 8;   // [NST]
+  const uint32_t b_vempty = bar0 + 16 * 8;  // [NST]
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 4);
+  float* s_xchg = reinterpret_cast<float*>(smem + kOffXchg);     // [2 halves][128 rows]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
+    mbar_init(b_qfull, 1);
+    mbar_init(b_qempty, 1);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(b_qfull + 8 * i, 1);
-      mbar_init(b_qempty + 8 * i, 1);
       mbar_init(b_sfull + 8 * i, 1);
-      mbar_init(b_sfree + 8 * i, 128);
+      mbar_init(b_sfree + 8 * i, kSoftmaxWarps * 32);
+      mbar_init(b_pfull + 8 * i, kSoftmaxWarps * 32);
+      mbar_init(b_pvdone + 8 * i, 1);
     }
     for (int i = 0; i < NST; ++i) {
-      mbar_init(b_kvfull + 8 * i, 1);
-      mbar_init(b_kvempty + 8 * i, 1);
+      mbar_init(b_kfull + 8 * i, 1);
+      mbar_init(b_kempty + 8 * i, 1);
+      mbar_init(b_vfull + 8 * i, 1);
+      mbar_init(b_vempty + 8 * i, 1);
     }
-    mbar_init(b_pfull, 128);
-    mbar_init(b_pvdone, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(s_tmem), kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_kpos);
     prefetch_tmap(&tm_vpos);
@@ -169,46 +186,49 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == kProducerWarp || warp == kVProducerWarp) {
+    // ------------------------------------------------------------ producers
+    // warp kProducerWarp: Q and K tiles; warp kVProducerWarp: V tiles.  Both
+    // walk the same item/tile sequence.
+    const bool is_k = (warp == kProducerWarp);
     if (lane == 0) {
+      const uint32_t ring = is_k ? sK : sV;
+      const uint32_t b_full = is_k ? b_kfull : b_vfull;
+      const uint32_t b_empty = is_k ? b_kempty : b_vempty;
       int g = 0, li = 0;
-      for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x, ++li) {
+      bool ok = true;
+      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
         const Item it = make_item(p, idx);
-        const int qb = li & 1;
-        if (li >= 2 && !mbar_wait(b_qempty + 8 * qb, ((li >> 1) - 1) & 1, s_abort)) break;
-        mbar_arrive_expect_tx(b_qfull + 8 * qb, kTile);
-        tma_load_4d(sQ + qb * kTile, &tm_q, b_qfull + 8 * qb, 0, it.h, it.t0, it.b);
-        tma_load_4d(sQ + qb * kTile + kHalf, &tm_q, b_qfull + 8 * qb, 64, it.h, it.t0, it.b);
-        bool ok = true;
+        if (is_k) {
+          if (li >= 1 && !mbar_wait(b_qempty, (li - 1) & 1, s_abort)) break;
+          mbar_arrive_expect_tx(b_qfull, kTile);
+          tma_load_4d(sQ, &tm_q, b_qfull, 0, it.h, it.t0, it.b);
+          tma_load_4d(sQ + kHalf, &tm_q, b_qfull, 64, it.h, it.t0, it.b);
+        }
         for (int j = 0; j < it.n_tiles; ++j, ++g) {
           const int st = g % NST;
-          if (g >= NST && !mbar_wait(b_kvempty + 8 * st, ((g / NST) - 1) & 1, s_abort)) {
+          if (g >= NST && !mbar_wait(b_empty + 8 * st, ((g / NST) - 1) & 1, s_abort)) {
             ok = false;
             break;
           }
-          const CUtensorMap* mk;
-          const CUtensorMap* mv;
+          const CUtensorMap* m;
           int row;
           if (j < it.n_win) {
-            mk = &tm_kpos; mv = &tm_vpos;
+            m = is_k ? &tm_kpos : &tm_vpos;
             row = it.p_start + j * BN;
           } else {
             row = (j - it.n_win) * BN;
-            if (it.dense) { mk = &tm_kpos; mv = &tm_vpos; }
-            else { mk = &tm_kdil; mv = &tm_vdil; }
+            if (it.dense) m = is_k ? &tm_kpos : &tm_vpos;
+            else m = is_k ? &tm_kdil : &tm_vdil;
           }
-          const uint32_t fb = b_kvfull + 8 * st;
-          mbar_arrive_expect_tx(fb, 2 * kTile);
-          tma_load_4d(sK + st * kTile, mk, fb, 0, it.h, row, it.b);
-          tma_load_4d(sK + st * kTile + kHalf, mk, fb, 64, it.h, row, it.b);
-          tma_load_4d(sV + st * kTile, mv, fb, 0, it.h, row, it.b);
-          tma_load_4d(sV + st * kTile + kHalf, mv, fb, 64, it.h, row, it.b);
+          const uint32_t fb = b_full + 8 * st;
+          mbar_arrive_expect_tx(fb, kTile);
+          tma_load_4d(ring + st * kTile, m, fb, 0, it.h, row, it.b);
+          tma_load_4d(ring + st * kTile + kHalf, m, fb, 64, it.h, row, it.b);
         }
-        if (!ok) break;
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);    // Q K^T: both K-major
@@ -218,37 +238,39 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       int pg = 0, pst = 0, pacc = 0;
       bool ok = true;
       auto issue_pv = [&](int gg, int stg, int acc) -> bool {
-        if (!mbar_wait(b_pfull, gg & 1, s_abort)) return false;
+        const int pb = gg & 1;
+        if (!mbar_wait(b_pfull + 8 * pb, (gg >> 1) & 1, s_abort)) return false;
+        if (!mbar_wait(b_vfull + 8 * stg, (gg / NST) & 1, s_abort)) return false;
         tc_fence_after();
 #pragma unroll
         for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t a = sw128_desc(sP + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
+          const uint64_t a = sw128_desc(sP + pb * kTile + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
           const uint64_t bdesc = sw128_desc(sV + stg * kTile + k * 16 * 128, kHalf, 1024);
           umma_f16(tmem + kColO, a, bdesc, idPV, (acc || k > 0) ? 1u : 0u);
         }
-        umma_commit(b_kvempty + 8 * stg);
-        umma_commit(b_pvdone);
+        umma_commit(b_vempty + 8 * stg);
+        umma_commit(b_pvdone + 8 * pb);
         return true;
       };
       for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
         const Item it = make_item(p, idx);
-        const int qb = li & 1;
-        if (!mbar_wait(b_qfull + 8 * qb, (li >> 1) & 1, s_abort)) { ok = false; break; }
+        if (!mbar_wait(b_qfull, li & 1, s_abort)) { ok = false; break; }
         for (int j = 0; j < it.n_tiles; ++j, ++g) {
           const int st = g % NST;
           const int sbuf = g & 1;
-          if (!mbar_wait(b_kvfull + 8 * st, (g / NST) & 1, s_abort)) { ok = false; break; }
+          if (!mbar_wait(b_kfull + 8 * st, (g / NST) & 1, s_abort)) { ok = false; break; }
           if (g >= 2 && !mbar_wait(b_sfree + 8 * sbuf, ((g >> 1) - 1) & 1, s_abort)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < DH / 16; ++k) {
             const uint32_t koff = (k >> 2) * kHalf + (k & 3) * 32;
-            const uint64_t a = sw128_desc(sQ + qb * kTile + koff, 16, 1024);
+            const uint64_t a = sw128_desc(sQ + koff, 16, 1024);
             const uint64_t bdesc = sw128_desc(sK + st * kTile + koff, 16, 1024);
             umma_f16(tmem + kColS + sbuf * BN, a, bdesc, idS, k > 0 ? 1u : 0u);
           }
           umma_commit(b_sfull + 8 * sbuf);
-          if (j == it.n_tiles - 1) umma_commit(b_qempty + 8 * qb);
+          umma_commit(b_kempty + 8 * st);
+          if (j == it.n_tiles - 1) umma_commit(b_qempty);
           if (pend && !issue_pv(pg, pst, pacc)) { ok = false; break; }
           pend = true;
           pg = g; pst = st; pacc = (j > 0);
@@ -259,11 +281,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = threadIdx.x;                       // query row within the tile
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const int r = (warp & 3) * 32 + lane;            // query row within the tile (TMEM lane)
+    const int half = warp >> 2;                      // key/output column half
+    const int c_base = half * 64;
+    const uint32_t bar_id = 1 + (warp & 3);          // named barrier of the warp pair
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    float* x_mine = s_xchg + half * BM + r;
+    const float* x_other = s_xchg + (1 - half) * BM + r;
+    auto pair_sync = [&]() {
+      asm volatile("bar.sync %0, %1;" :: "r"(bar_id), "r"(64) : "memory");
+    };
+    // The two warps of a pair meet at named barriers, so neither may leave the
+    // schedule early: after a failed (timed-out or aborted) wait the warps
+    // carry on with whatever tensor memory holds; every later wait fails fast
+    // and the error word already records the timeout.
     int g = 0;
-    bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
       const Item it = make_item(p, idx);
       const int t = it.t0 + r;
       const bool row_ok = t < p.T;
@@ -272,92 +305,149 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       float m_used = -1e30f, l = 0.f;
       for (int j = 0; j < it.n_tiles; ++j, ++g) {
         const int sbuf = g & 1;
-        if (!warp_all(mbar_wait(b_sfull + 8 * sbuf, (g >> 1) & 1, s_abort))) { ok = false; break; }
+        warp_all(mbar_wait(b_sfull + 8 * sbuf, (g >> 1) & 1, s_abort));
         tc_fence_after();
-        uint32_t sr[BN];
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) tmem_ld32(tl + kColS + sbuf * BN + c * 32, sr + c * 32);
+        uint32_t sr[64];
+        tmem_ld32(tl + kColS + sbuf * BN + c_base, sr);
+        tmem_ld32(tl + kColS + sbuf * BN + c_base + 32, sr + 32);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(b_sfree + 8 * sbuf);
 
-        float x[BN];
-        float mx = -INFINITY;
+        // validity bit masks of the two 32-column chunks of this half
+        uint32_t vm[2];
         if (j < it.n_win) {
-          const int p0 = it.p_start + j * BN;
-          int rm = p0 % it.Dd;
+          const int p0 = it.p_start + j * BN + c_base;       // position of column 0 of the half
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const int pos = p0 + c;
-            const bool dup = (rm == it.Dd - 1) && (pos < t);
-            const bool ok_c = (pos >= w_lo) && (pos <= t) && !dup;
-            x[c] = ok_c ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[c]);
-            rm = (rm + 1 == it.Dd) ? 0 : rm + 1;
+          for (int k = 0; k < 2; ++k) {
+            const int cb = p0 + 32 * k;
+            const int lo = min(max(w_lo - cb, 0), 32);         // first valid bit
+            const int hi = min(max(t - cb + 1, 0), 32);        // one past the last valid bit
+            uint32_t m = (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~(lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u));
+            // keys already in the dilated set: positions q = D-1 (mod D), q < t
+            const int lim = min(max(t - cb, 0), 32);
+            int i0 = (it.Dd - 1) - (cb % it.Dd);
+            if (i0 < 0) i0 += it.Dd;
+            for (int i = i0; i < lim; i += it.Dd) m &= ~(1u << i);
+            vm[k] = m;
           }
         } else {
-          const int lim = lim_dil - (j - it.n_win) * BN;
+          const int lim = lim_dil - (j - it.n_win) * BN - c_base;
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            x[c] = (c < lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, x[c]);
+          for (int k = 0; k < 2; ++k) {
+            const int n = min(max(lim - 32 * k, 0), 32);
+            vm[k] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
           }
         }
-        // previous P.V must be complete before P is overwritten / O rescaled
-        if (g > 0 && !warp_all(mbar_wait(b_pvdone, (g - 1) & 1, s_abort))) { ok = false; break; }
-        tc_fence_after();
-        // O is rescaled only when some row's running max grew by more than
-        // 2^kRescaleThreshold.  tcgen05.ld/st are warp-collective, so the
-        // decision is taken per warp and rows that do not need it use alpha 1.
-        const bool need = (j > 0) && (mx > m_used + kRescaleThreshold);
-        if (j == 0) m_used = fmaxf(mx, -1e30f);
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? exp2f(m_used - mx) : 1.f;
+        // masked row max of this half (raw scores)
+        // (four independent accumulators per chunk keep the chain short)
+        float mx = -INFINITY;
 #pragma unroll
-          for (int c = 0; c < DH / 32; ++c) {
+        for (int k = 0; k < 2; ++k) {
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (vm[k] == 0xffffffffu) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sr[32 * k + i]));
+          } else if (vm[k] != 0u) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float v = __uint_as_float(sr[32 * k + i]);
+              m4[i & 3] = fmaxf(m4[i & 3], ((vm[k] >> i) & 1u) ? v : -INFINITY);
+            }
+          }
+          mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+        }
+        // combine with the partner half of the row
+        *x_mine = mx;
+        pair_sync();
+        mx = fmaxf(mx, *x_other);
+        pair_sync();
+        const float mxs = mx * p.scale_log2;               // -inf stays -inf
+        // P buffer g&1 was last read by P.V of tile g-2
+        if (g >= 2) warp_all(mbar_wait(b_pvdone + 8 * sbuf, ((g >> 1) - 1) & 1, s_abort));
+        // O is rescaled only when some row's running max grew by more than
+        // 2^kRescaleThreshold; tcgen05.ld/st are warp-collective, so the
+        // decision is per warp (both warps of a pair decide alike) and rows
+        // that do not need it scale by 1.  P.V of tile g-1 must be complete.
+        const bool need = (j > 0) && (mxs > m_used + kRescaleThreshold);
+        if (j == 0) m_used = fmaxf(mxs, -1e30f);
+        if (__any_sync(0xffffffffu, need)) {
+          const int pb1 = (g - 1) & 1;
+          warp_all(mbar_wait(b_pvdone + 8 * pb1, ((g - 1) >> 1) & 1, s_abort));
+          tc_fence_after();
+          const float alpha = need ? exp2f(m_used - mxs) : 1.f;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
             uint32_t o32[32];
-            tmem_ld32(tl + kColO + c * 32, o32);
+            tmem_ld32(tl + kColO + c_base + c * 32, o32);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
-            tmem_st32(tl + kColO + c * 32, o32);
+            tmem_st32(tl + kColO + c_base + c * 32, o32);
           }
           tmem_wait_st();
           if (need) {
             l *= alpha;
-            m_used = mx;
+            m_used = mxs;
           }
         }
-        float rowsum = 0.f;
+        // p = 2^(s*scale - m), bf16 into the swizzled P tile (keys c_base..c_base+63)
+        const uint32_t prow = sP + sbuf * kTile + half * kHalf + r * 128;
+        const float neg_m = -m_used;
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int cc = 0; cc < BN / 8; ++cc) {
-          uint32_t w[4];
+        for (int k = 0; k < 2; ++k) {
+          uint32_t w[16];
+          if (vm[k] == 0u) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float e0 = exp2f(x[cc * 8 + 2 * i] - m_used);
-            const float e1 = exp2f(x[cc * 8 + 2 * i + 1] - m_used);
-            w[i] = pack_bf16x2(e0, e1);
-            rowsum += __uint_as_float(w[i] << 16) + __uint_as_float(w[i] & 0xffff0000u);
+            for (int i = 0; i < 16; ++i) w[i] = 0u;
+          } else if (vm[k] == 0xffffffffu) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float e0 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i]), p.scale_log2, neg_m));
+              const float e1 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i + 1]), p.scale_log2, neg_m));
+              rs[i & 3] += e0 + e1;
+              w[i] = pack_bf16x2(e0, e1);
+            }
+          } else {
+            // exponentiate every column, then select: no per-element branches
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float e0 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i]), p.scale_log2, neg_m));
+              float e1 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i + 1]), p.scale_log2, neg_m));
+              e0 = ((vm[k] >> (2 * i)) & 1u) ? e0 : 0.f;
+              e1 = ((vm[k] >> (2 * i + 1)) & 1u) ? e1 : 0.f;
+              rs[i & 3] += e0 + e1;
+              w[i] = pack_bf16x2(e0, e1);
+            }
           }
-          const uint32_t addr = sP + (cc >> 3) * kHalf + r * 128 + ((((uint32_t)cc & 7u) ^ ((uint32_t)r & 7u)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                       :: "r"(addr), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]) : "memory");
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint32_t chunk = (uint32_t)(4 * k + v);                 // 16-byte chunk in the half row
+            const uint32_t addr = prow + ((chunk ^ ((uint32_t)r & 7u)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                         :: "r"(addr), "r"(w[4 * v]), "r"(w[4 * v + 1]), "r"(w[4 * v + 2]), "r"(w[4 * v + 3])
+                         : "memory");
+          }
         }
-        l += rowsum;
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
         fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(b_pfull);
+        mbar_arrive(b_pfull + 8 * sbuf);
       }
-      if (!ok) break;
-      // ---- epilogue: O / l -> bf16 -> global
-      if (!warp_all(mbar_wait(b_pvdone, (g - 1) & 1, s_abort))) { ok = false; break; }
+      // ---- epilogue: O / l -> bf16 -> global (each thread half a row)
+      const int gl = g - 1;
+      warp_all(mbar_wait(b_pvdone + 8 * (gl & 1), (gl >> 1) & 1, s_abort));
       tc_fence_after();
-      const float inv = 1.f / l;
-      __nv_bfloat16* orow = p.o + (((size_t)it.b * p.T + t) * p.H + it.h) * DH;
+      *x_mine = l;
+      pair_sync();
+      const float inv = 1.f / (l + *x_other);
+      pair_sync();
+      __nv_bfloat16* orow = p.o + (((size_t)it.b * p.T + t) * p.H + it.h) * DH + c_base;
 #pragma unroll
-      for (int c = 0; c < DH / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t o32[32];
-        tmem_ld32(tl + kColO + c * 32, o32);
+        tmem_ld32(tl + kColO + c_base + c * 32, o32);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
@@ -377,7 +467,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

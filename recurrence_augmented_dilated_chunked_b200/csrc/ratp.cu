@@ -280,24 +280,32 @@ struct CacheLayout {
   int max_splits, split_keys;
 };
 
-constexpr int kDefaultSplitKeys = 256;
+// Decode grid sizing: keys per split chosen so that one step is about one
+// wave of CTAs (kDecodeCtasPerSm resident per SM), never below kMinSplitKeys.
+constexpr int kDecodeCtasPerSm = 6;
+constexpr int kMinSplitKeys = 128;
 
 int cache_layout(int B, int H, int Dh, int T_max, int D, int W, const uint8_t* head_mask,
                  CacheLayout* L) {
   if (B < 1 || H < 1 || T_max < 1 || D < 1 || W < 0) return RATP_ERR_ARG;
   if (Dh != 128 && Dh != 64) return RATP_ERR_SHAPE;
   if (H > RATP_MAX_HEADS) return RATP_ERR_SHAPE;
-  long long per_b = 0;
+  long long per_b = 0, keys_total = 0;
   int max_keys = 0;
   for (int h = 0; h < H; ++h) {
     const bool dense = head_mask != nullptr && head_mask[h] != 0;
     const int cap = dense ? T_max : T_max / D;
     per_b += cap;
     const int keys = cap + (dense ? 0 : W);
+    keys_total += (long long)B * keys;
     if (keys > max_keys) max_keys = keys;
   }
   L->rows_per_b = per_b;
-  L->split_keys = kDefaultSplitKeys;
+  const long long target_ctas = (long long)sm_count() * kDecodeCtasPerSm;
+  long long split = (keys_total + target_ctas - 1) / target_ctas;
+  if (split < kMinSplitKeys) split = kMinSplitKeys;
+  if (split > (1 << 30)) split = 1 << 30;
+  L->split_keys = (int)split;
   L->max_splits = (max_keys + L->split_keys - 1) / L->split_keys;
   if (L->max_splits < 1) L->max_splits = 1;
   const size_t row_bytes = (size_t)Dh * 2;

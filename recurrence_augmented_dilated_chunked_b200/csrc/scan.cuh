@@ -13,13 +13,16 @@
 //     channels with 16-byte vectors, so every load instruction of a warp reads
 //     whole 128-byte lines; each thread holds R = 4 consecutive tokens.
 //   * in registers: each thread reduces its 4 tokens to one affine map; the
-//     row groups of the CTA are combined by a shuffle scan in shared memory.
+//     row groups of a warp are combined by a shuffle scan, the 8 warp totals
+//     by one warp through shared memory.
 //   * across chunks: decoupled look-back.  Chunk tickets come from an atomic
 //     counter in launch order, so a CTA only waits on chunks whose CTAs have
-//     started.  A CTA publishes its aggregate map at once, then warp 0 polls
-//     up to 32 predecessors in parallel and composes their aggregates until it
-//     meets a published inclusive state.  Inputs stay in registers while it
-//     waits, so x and g are read from HBM exactly once.
+//     started.  Each lane of warp 0 owns two channels of the chunk's
+//     descriptor: it publishes its part of the aggregate map at once (its own
+//     release flag), then polls 4 predecessors at a time and composes their
+//     aggregates until it meets a published inclusive state.  The chunk stays
+//     in shared memory (TMA-filled) while it waits, so x and g are read from
+//     HBM exactly once.
 //   * every wait is bounded (kSpinTimeoutNs); on expiry the kernel records
 //     RATP_ERR_TIMEOUT and finishes with a zero carry.
 #pragma once
@@ -43,7 +46,7 @@ struct Shape {
 
 // Workspace layout (bytes), given n = total chunks and NS streams:
 //   [0, 256)                ticket counter (u32)
-//   flags  u32 [n]          0 empty, 1 aggregate ready, 2 inclusive ready
+//   flags  u32 [n][32]      per publishing lane: 0 empty, 1 aggregate, 2 inclusive
 //   agg    f32 [n][1+NS][64] aggregate map (a, b_stream...)
 //   incl   f32 [n][NS][64]   inclusive state at the chunk's last token
 struct Workspace {
@@ -55,9 +58,11 @@ struct Workspace {
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+constexpr int kFlagLanes = 32;   // lane l of warp 0 publishes channels 2l, 2l+1
+
 inline size_t workspace_bytes(long long n_chunks, int NS) {
   size_t b = 256;
-  b += align256(sizeof(unsigned int) * n_chunks);
+  b += align256(sizeof(unsigned int) * kFlagLanes * n_chunks);
   b += align256(sizeof(float) * n_chunks * (1 + NS) * kSlab);
   b += align256(sizeof(float) * n_chunks * NS * kSlab);
   return b;
@@ -69,7 +74,7 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
   w.counter = reinterpret_cast<unsigned int*>(p);
   p += 256;
   w.flags = reinterpret_cast<unsigned int*>(p);
-  p += align256(sizeof(unsigned int) * n_chunks);
+  p += align256(sizeof(unsigned int) * kFlagLanes * n_chunks);
   w.agg = reinterpret_cast<float*>(p);
   p += align256(sizeof(float) * n_chunks * (1 + NS) * kSlab);
   w.incl = reinterpret_cast<float*>(p);
@@ -78,7 +83,7 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
 
 // Bytes to zero before each launch: counter + flags.
 inline size_t reset_bytes(long long n_chunks) {
-  return 256 + align256(sizeof(unsigned int) * n_chunks);
+  return 256 + align256(sizeof(unsigned int) * kFlagLanes * n_chunks);
 }
 
 template <typename T, int NS>
@@ -98,58 +103,30 @@ template <typename T, int NS>
 struct Smem {
   static constexpr int kTile = Shape<T>::kChunk * kSlab * (int)sizeof(T);   // 16 KB
   static constexpr int kData = (1 + NS) * kTile;
-  static constexpr int kScan = Shape<T>::kGroups * kSlab * (1 + NS) * 4;
+  // per-warp totals of the intra-chunk scan: [warps][1 + NS][kSlab] floats
+  static constexpr int kScan = (kThreads / 32) * (1 + NS) * kSlab * 4;
   static constexpr int kBytes = kData + kScan + 128;                       // + alignment
 };
 
-// Compose the affine maps of up to 8 predecessor chunks (nearest first) into
-// the running composite x -> ca*x + cb, with all loads issued before use.
-template <int NS>
-__device__ __forceinline__ void compose_batch(const float* agg, long long d0, int n, int c0,
-                                              float& ca0, float& ca1, float (&cb0)[NS],
-                                              float (&cb1)[NS]) {
-  float2 pa[8], pb[NS][8];
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    if (u < n) {
-      const float* src = agg + (d0 - u) * (1 + NS) * kSlab;
-      pa[u] = __ldcg(reinterpret_cast<const float2*>(src + c0));
-#pragma unroll
-      for (int s = 0; s < NS; ++s) pb[s][u] = __ldcg(reinterpret_cast<const float2*>(src + (1 + s) * kSlab + c0));
-    }
-  }
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    if (u < n) {
-#pragma unroll
-      for (int s = 0; s < NS; ++s) {
-        cb0[s] = fmaf(ca0, pb[s][u].x, cb0[s]);
-        cb1[s] = fmaf(ca1, pb[s][u].y, cb1[s]);
-      }
-      ca0 *= pa[u].x;
-      ca1 *= pa[u].y;
-    }
-  }
-}
-
 template <typename T, int NS>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 4)
 scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x0,
             const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ Params<T, NS> p) {
   using S = Shape<T>;
   using SM = Smem<T, NS>;
-  constexpr int V = S::kVec, LANES = S::kLanes, G = S::kGroups, L = S::kChunk;
+  constexpr int V = S::kVec, LANES = S::kLanes, L = S::kChunk;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const T* s_g = reinterpret_cast<const T*>(smem);
-  float* s_a = reinterpret_cast<float*>(smem + SM::kData);            // [G][64]
-  float* s_b = s_a + G * kSlab;                                        // [NS][G][64]
+  constexpr int NW = kThreads / 32;
+  float* s_w = reinterpret_cast<float*>(smem + SM::kData);            // [NW][1 + NS][64]
   __shared__ __align__(8) uint64_t s_bar;
   __shared__ unsigned int s_ticket;
   __shared__ float s_tot_a[kSlab];
   __shared__ float s_tot_b[NS][kSlab];
   __shared__ float s_carry[NS][kSlab];
+  static_assert(32 % LANES == 0, "row groups of a warp must share channels");
 
   const int tid = threadIdx.x;
   const uint32_t bar = sm100::smem_u32(&s_bar);
@@ -193,13 +170,11 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     if (!__syncthreads_and(ok)) {
       // publish a zero state so that successors do not wait on this chunk
       if (tid < 32) {
-        for (int i = tid; i < NS * kSlab; i += 32) __stcg(p.ws.incl + desc * NS * kSlab + i, 0.f);
-        __threadfence();
-        __syncwarp();
-        if (tid == 0) {
-          raise_error(RATP_ERR_TIMEOUT);
-          st_release_gpu(p.ws.flags + (long long)chain * p.n_chunks_t + chunk, 2u);
-        }
+#pragma unroll
+        for (int s = 0; s < NS; ++s)
+          __stcg(reinterpret_cast<float2*>(p.ws.incl + (desc * NS + s) * kSlab + 2 * tid), make_float2(0.f, 0.f));
+        st_release_gpu(p.ws.flags + desc * kFlagLanes + tid, 2u);
+        if (tid == 0) raise_error(RATP_ERR_TIMEOUT);
       }
       return;
     }
@@ -229,75 +204,119 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
       for (int i = 0; i < V; ++i) la[i] *= gf[i];
     }
   }
+  // ---- intra-chunk scan over row groups, hierarchical ----
+  // (1) the row groups of one warp hold the same channels in lanes
+  //     lane_c, lane_c + LANES, ...: a shuffle scan over them (stride LANES)
+  //     gives each thread the map of the warp's rows up to and including its
+  //     own; (2) lane group GW-1 publishes the warp total, warp 0 scans the NW
+  //     totals per channel; (3) each thread composes the exclusive prefix.
+  constexpr int GW = 32 / LANES;             // row groups per warp
+  const int lane = tid & 31, wid = tid >> 5;
+  const int gw = lane / LANES;               // row group within the warp
+  float ia[V], ib[NS][V];                    // inclusive map within the warp
 #pragma unroll
   for (int i = 0; i < V; ++i) {
-    s_a[grp * kSlab + lane_c * V + i] = la[i];
+    ia[i] = la[i];
 #pragma unroll
-    for (int s = 0; s < NS; ++s) s_b[(s * G + grp) * kSlab + lane_c * V + i] = lb[s][i];
+    for (int s = 0; s < NS; ++s) ib[s][i] = lb[s][i];
   }
-  __syncthreads();
-
-  // ---- exclusive scan over the G row groups, per channel (shuffle scan) ----
-  {
-    constexpr int kBlocks = kThreads / G;          // channel blocks
-    const int gi = tid % G;                        // row group handled
-    const int cb = tid / G;
-    for (int c = cb; c < kSlab; c += kBlocks) {
-      float a = s_a[gi * kSlab + c];
-      float bb[NS];
 #pragma unroll
-      for (int s = 0; s < NS; ++s) bb[s] = s_b[(s * G + gi) * kSlab + c];
+  for (int d = 1; d < GW; d <<= 1) {
 #pragma unroll
-      for (int d = 1; d < G; d <<= 1) {
-        const float ua = __shfl_up_sync(0xffffffffu, a, d, G);
-        float ub[NS];
+    for (int i = 0; i < V; ++i) {
+      const float ua = __shfl_up_sync(0xffffffffu, ia[i], d * LANES);
+      float ub[NS];
 #pragma unroll
-        for (int s = 0; s < NS; ++s) ub[s] = __shfl_up_sync(0xffffffffu, bb[s], d, G);
-        if (gi >= d) {
+      for (int s = 0; s < NS; ++s) ub[s] = __shfl_up_sync(0xffffffffu, ib[s][i], d * LANES);
+      if (gw >= d) {
 #pragma unroll
-          for (int s = 0; s < NS; ++s) bb[s] = fmaf(a, ub[s], bb[s]);   // self o up
-          a *= ua;
-        }
+        for (int s = 0; s < NS; ++s) ib[s][i] = fmaf(ia[i], ub[s], ib[s][i]);   // self o up
+        ia[i] *= ua;
       }
-      float ea = __shfl_up_sync(0xffffffffu, a, 1, G);
-      float eb[NS];
+    }
+  }
+  if (gw == GW - 1) {                        // warp total
 #pragma unroll
-      for (int s = 0; s < NS; ++s) eb[s] = __shfl_up_sync(0xffffffffu, bb[s], 1, G);
-      if (gi == 0) {
-        ea = 1.f;
+    for (int i = 0; i < V; ++i) {
+      s_w[(wid * (1 + NS)) * kSlab + lane_c * V + i] = ia[i];
 #pragma unroll
-        for (int s = 0; s < NS; ++s) eb[s] = 0.f;
-      }
-      if (gi == G - 1) {
-        s_tot_a[c] = a;
-#pragma unroll
-        for (int s = 0; s < NS; ++s) s_tot_b[s][c] = bb[s];
-      }
-      s_a[gi * kSlab + c] = ea;
-#pragma unroll
-      for (int s = 0; s < NS; ++s) s_b[(s * G + gi) * kSlab + c] = eb[s];
+      for (int s = 0; s < NS; ++s) s_w[(wid * (1 + NS) + 1 + s) * kSlab + lane_c * V + i] = ib[s][i];
     }
   }
   __syncthreads();
+  if (tid < 32) {
+    // exclusive prefix over warps (in place) and the chunk total, 2 channels per lane
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+      const int c = 2 * tid + cc;
+      float pa = 1.f, pb[NS];
+#pragma unroll
+      for (int s = 0; s < NS; ++s) pb[s] = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float wa = s_w[(w * (1 + NS)) * kSlab + c];
+        float wb[NS];
+#pragma unroll
+        for (int s = 0; s < NS; ++s) wb[s] = s_w[(w * (1 + NS) + 1 + s) * kSlab + c];
+        s_w[(w * (1 + NS)) * kSlab + c] = pa;
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          s_w[(w * (1 + NS) + 1 + s) * kSlab + c] = pb[s];
+          pb[s] = fmaf(wa, pb[s], wb[s]);    // warp w applied after the prefix
+        }
+        pa *= wa;
+      }
+      s_tot_a[c] = pa;
+#pragma unroll
+      for (int s = 0; s < NS; ++s) s_tot_b[s][c] = pb[s];
+    }
+  }
+  __syncthreads();
+  // exclusive map of this thread's row group: (inclusive within warp minus
+  // own group) composed after the warp prefix
+  float ea[V], eb[NS][V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    // within-warp exclusive = the inclusive map of the row group above (gw - 1)
+    float xa = __shfl_up_sync(0xffffffffu, ia[i], LANES);
+    float xb[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) xb[s] = __shfl_up_sync(0xffffffffu, ib[s][i], LANES);
+    if (gw == 0) {
+      xa = 1.f;
+#pragma unroll
+      for (int s = 0; s < NS; ++s) xb[s] = 0.f;
+    }
+    const float wa = s_w[(wid * (1 + NS)) * kSlab + lane_c * V + i];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const float wb = s_w[(wid * (1 + NS) + 1 + s) * kSlab + lane_c * V + i];
+      eb[s][i] = fmaf(xa, wb, xb[s]);        // (within-warp exclusive) o (warp prefix)
+    }
+    ea[i] = xa * wa;
+  }
 
   // ---- publish, look back, publish inclusive (warp 0) ----
+  // Lane l of warp 0 owns channels 2l, 2l+1 of the chunk descriptors: it
+  // writes them and then releases its own flag, and in a successor chunk the
+  // lane with the same index acquires that flag before reading them.  Every
+  // release/acquire pair is thread-to-thread, so no fence is needed.
   if (tid < 32) {
     const int lane = tid;
-    unsigned int* flags = p.ws.flags + (long long)chain * p.n_chunks_t;
+    const unsigned int* cflags = p.ws.flags + (long long)chain * p.n_chunks_t * kFlagLanes + lane;
+    unsigned int* my_flag = p.ws.flags + desc * kFlagLanes + lane;
     const float* agg = p.ws.agg;
     float* incl = p.ws.incl;
-    const int c0 = lane * 2;                  // two channels per lane
+    const int c0 = lane * 2;
+    float cb0[NS], cb1[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
     if (chunk == 0) {
 #pragma unroll
-      for (int s = 0; s < NS; ++s) {
-        s_carry[s][c0] = 0.f;
-        s_carry[s][c0 + 1] = 0.f;
+      for (int s = 0; s < NS; ++s)
         __stcg(reinterpret_cast<float2*>(incl + (desc * NS + s) * kSlab + c0),
                make_float2(s_tot_b[s][c0], s_tot_b[s][c0 + 1]));
-      }
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release_gpu(flags + chunk, 2u);
+      st_release_gpu(my_flag, 2u);
     } else {
       {
         float* dst = p.ws.agg + desc * (1 + NS) * kSlab;
@@ -307,83 +326,99 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
           __stcg(reinterpret_cast<float2*>(dst + (1 + s) * kSlab + c0),
                  make_float2(s_tot_b[s][c0], s_tot_b[s][c0 + 1]));
       }
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release_gpu(flags + chunk, 1u);
+      st_release_gpu(my_flag, 1u);
 
-      // composite map of the predecessors seen so far: x -> ca x + cb
+      // composite map of the predecessors composed so far: x -> ca x + cb
       float ca0 = 1.f, ca1 = 1.f;
-      float cb0[NS], cb1[NS];
-#pragma unroll
-      for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
-      int top = chunk - 1;                     // nearest predecessor not yet composed
+      int top = chunk - 1;                      // nearest predecessor not yet composed
       const unsigned long long t_start = global_ns();
       while (true) {
-        const int k = top - lane;
-        const unsigned int f = (k >= 0) ? ld_acquire_gpu(flags + k) : 3u;   // 3: before start
-        const unsigned int incl_mask = __ballot_sync(0xffffffffu, f >= 2u);
-        const unsigned int empty_mask = __ballot_sync(0xffffffffu, f == 0u);
-        int upto = -1;                          // compose lanes [0, upto)
-        bool found = false;
-        if (incl_mask != 0u) {
-          const int jl = __ffs(incl_mask) - 1;
-          const unsigned int below = (jl == 0) ? 0u : ((1u << jl) - 1u);
-          if ((empty_mask & below) == 0u) { upto = jl; found = true; }
-        } else if (empty_mask == 0u) {
-          upto = 32;                            // 32 aggregates: compose, go further back
+        constexpr int kWin = 4;                 // predecessors polled at once
+        const int n = min(kWin, top + 1);
+        unsigned int f[kWin];
+#pragma unroll
+        for (int u = 0; u < kWin; ++u) f[u] = (u < n) ? ld_acquire_gpu(cflags + (long long)(top - u) * kFlagLanes) : 0u;
+        int upto = -1;                          // aggregates to compose
+        bool found = false;                     // an inclusive state ends the walk
+#pragma unroll
+        for (int u = kWin - 1; u >= 0; --u) {   // nearest inclusive with no gap before it
+          if (u < n && f[u] >= 2u) { upto = u; found = true; }
+        }
+        if (found) {
+#pragma unroll
+          for (int u = 0; u < kWin; ++u)
+            if (u < upto && f[u] == 0u) found = false;
+          if (!found) upto = -1;
+        } else {
+          bool all = true;
+#pragma unroll
+          for (int u = 0; u < kWin; ++u)
+            if (u < n && f[u] == 0u) all = false;
+          if (all) upto = n;
         }
         if (upto < 0) {
-          const bool expired = (global_ns() - t_start) > kSpinTimeoutNs;
-          if (__any_sync(0xffffffffu, expired)) {
-            if (lane == 0) raise_error(RATP_ERR_TIMEOUT);
+          if (global_ns() - t_start > kSpinTimeoutNs) {
+            raise_error(RATP_ERR_TIMEOUT);
             ca0 = ca1 = 0.f;                     // give up: zero carry
 #pragma unroll
             for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
             break;
           }
-          __nanosleep(32);
+          __nanosleep(20);
           continue;
         }
-        __syncwarp();
-        __threadfence();
-        // inclusive state of the chunk that ends the look-back (issued first)
-        float v0[NS], v1[NS];
+        // all data loads of this window are issued before they are used
+        float2 pa[kWin], pb[NS][kWin], pv[NS];
 #pragma unroll
-        for (int s = 0; s < NS; ++s) { v0[s] = 0.f; v1[s] = 0.f; }
-        const int kin = top - upto;
-        if (found && kin >= 0) {
-          const long long dk = (long long)chain * p.n_chunks_t + kin;
+        for (int u = 0; u < kWin; ++u) {
+          if (u < upto) {
+            const float* src = agg + ((long long)chain * p.n_chunks_t + (top - u)) * (1 + NS) * kSlab;
+            pa[u] = __ldcg(reinterpret_cast<const float2*>(src + c0));
 #pragma unroll
-          for (int s = 0; s < NS; ++s) {
-            const float2 pv = __ldcg(reinterpret_cast<const float2*>(incl + (dk * NS + s) * kSlab + c0));
-            v0[s] = pv.x; v1[s] = pv.y;
+            for (int s = 0; s < NS; ++s) pb[s][u] = __ldcg(reinterpret_cast<const float2*>(src + (1 + s) * kSlab + c0));
           }
         }
-        const long long dtop = (long long)chain * p.n_chunks_t + top;
-        for (int m0 = 0; m0 < upto; m0 += 8)
-          compose_batch<NS>(agg, dtop - m0, min(8, upto - m0), c0, ca0, ca1, cb0, cb1);
+        if (found) {
+          const long long dk = (long long)chain * p.n_chunks_t + (top - upto);
+#pragma unroll
+          for (int s = 0; s < NS; ++s) pv[s] = __ldcg(reinterpret_cast<const float2*>(incl + (dk * NS + s) * kSlab + c0));
+        }
+#pragma unroll
+        for (int u = 0; u < kWin; ++u) {
+          if (u < upto) {
+#pragma unroll
+            for (int s = 0; s < NS; ++s) {
+              cb0[s] = fmaf(ca0, pb[s][u].x, cb0[s]);
+              cb1[s] = fmaf(ca1, pb[s][u].y, cb1[s]);
+            }
+            ca0 *= pa[u].x;
+            ca1 *= pa[u].y;
+          }
+        }
         if (found) {
 #pragma unroll
           for (int s = 0; s < NS; ++s) {
-            cb0[s] = fmaf(ca0, v0[s], cb0[s]);   // carry = composite(inclusive)
-            cb1[s] = fmaf(ca1, v1[s], cb1[s]);
+            cb0[s] = fmaf(ca0, pv[s].x, cb0[s]);   // carry = composite(inclusive)
+            cb1[s] = fmaf(ca1, pv[s].y, cb1[s]);
           }
           break;
         }
-        top -= 32;
+        top -= upto;
+        if (top < 0) break;                      // walked back to the sequence start
       }
-      // cb now holds the state entering this chunk
+      // cb now holds the state entering this chunk; publish the inclusive state
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        s_carry[s][c0] = cb0[s];
-        s_carry[s][c0 + 1] = cb1[s];
         const float e0 = fmaf(s_tot_a[c0], cb0[s], s_tot_b[s][c0]);
         const float e1 = fmaf(s_tot_a[c0 + 1], cb1[s], s_tot_b[s][c0 + 1]);
         __stcg(reinterpret_cast<float2*>(incl + (desc * NS + s) * kSlab + c0), make_float2(e0, e1));
       }
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) st_release_gpu(flags + chunk, 2u);
+      st_release_gpu(my_flag, 2u);
+    }
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      s_carry[s][c0] = cb0[s];
+      s_carry[s][c0 + 1] = cb1[s];
     }
   }
   __syncthreads();
@@ -393,9 +428,8 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
 #pragma unroll
   for (int i = 0; i < V; ++i) {
     const int c = lane_c * V + i;
-    const float ea = s_a[grp * kSlab + c];
 #pragma unroll
-    for (int s = 0; s < NS; ++s) hs[s][i] = fmaf(ea, s_carry[s][c], s_b[(s * G + grp) * kSlab + c]);
+    for (int s = 0; s < NS; ++s) hs[s][i] = fmaf(ea[i], s_carry[s][c], eb[s][i]);
   }
 #pragma unroll
   for (int r = 0; r < kRows; ++r) {
