@@ -84,9 +84,10 @@ int ratp_device_sm_count(int* sms);
  *   tensor (g is read once): hk = scan(xk, g), hv = scan(xv, g).
  *   final_state (nullable): fp32 [2][B][H][Dh] (k then v) -- the layout of the
  *   decode state.
- * workspace: device scratch of at least ratp_scan_workspace_bytes; it is
- *   re-initialised on `stream` by every call, so calls sharing one workspace
- *   must be ordered on one stream.  h may alias x (in-place) only when
+ * workspace: device scratch of at least ratp_scan_workspace_bytes.  It must
+ *   be zero-filled once before its first use; every call leaves it valid for
+ *   the next one (each launch tags its chunk descriptors with a fresh launch
+ *   number), and calls sharing one workspace must be ordered on one stream.  h may alias x (in-place) only when
  *   T == 1.  Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of
  *   64), ALIGN, CAPACITY (workspace too small).  T == 0 or B == 0 is a no-op.
  * ---------------------------------------------------------------------- */

@@ -130,7 +130,7 @@ def scan_workspace(B, T, H, Dh, dtype, device) -> torch.Tensor:
     key = (str(device), n.value)
     ws = _ws_cache.get(key)
     if ws is None:
-        ws = torch.empty(max(n.value, 256), dtype=torch.uint8, device=device)
+        ws = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=device)   # zero before first use
         _ws_cache[key] = ws
     return ws
 

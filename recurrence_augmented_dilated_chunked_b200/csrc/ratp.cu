@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -99,6 +100,15 @@ bool make_scan_map(CUtensorMap* m, const void* base, int B, int Tn, int C, int r
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Launch tags of the scan's self-validating chunk descriptors: unique per
+// launch within the process, never 0 (the value of a zero-filled workspace).
+std::atomic<unsigned int> g_scan_epoch{0};
+unsigned int next_scan_epoch() {
+  unsigned int e = ++g_scan_epoch;
+  while (e == 0) e = ++g_scan_epoch;
+  return e;
+}
+
 template <typename T, int NS>
 int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
                 int B, int Tn, int H, int Dh, const ScanGeom& geo,
@@ -110,6 +120,7 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   for (int s = 0; s < NS; ++s) p.h[s] = static_cast<T*>(h[s]);
   p.final_state = fs;
   p.ws = scan::carve(ws, geo.n_chunks, NS);
+  p.epoch = next_scan_epoch();
   p.B = B; p.Tn = Tn; p.C = H * Dh;
   p.slabs = geo.slabs; p.n_chains = geo.n_chains; p.n_chunks_t = geo.n_chunks_t;
   const int C = H * Dh, rows = scan::Shape<T>::kChunk;

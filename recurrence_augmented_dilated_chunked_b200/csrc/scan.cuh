@@ -18,9 +18,9 @@
 //   * across chunks: decoupled look-back.  Chunk tickets come from an atomic
 //     counter in launch order, so a CTA only waits on chunks whose CTAs have
 //     started.  Each lane of warp 0 owns two channels of the chunk's
-//     descriptor: it publishes its part of the aggregate map at once (its own
-//     release flag), then polls 4 predecessors at a time and composes their
-//     aggregates until it meets a published inclusive state.  The chunk stays
+//     descriptor: it publishes its part of the aggregate map at once as
+//     epoch-tagged 64-bit words, then reads two predecessors per round trip
+//     and composes their aggregates until it meets an inclusive state.  The chunk stays
 //     in shared memory (TMA-filled) while it waits, so x and g are read from
 //     HBM exactly once.
 //   * every wait is bounded (kSpinTimeoutNs); on expiry the kernel records
@@ -45,26 +45,28 @@ struct Shape {
 };
 
 // Workspace layout (bytes), given n = total chunks and NS streams:
-//   [0, 256)                ticket counter (u32)
-//   flags  u32 [n][32]      per publishing lane: 0 empty, 1 aggregate, 2 inclusive
-//   agg    f32 [n][1+NS][64] aggregate map (a, b_stream...)
-//   incl   f32 [n][NS][64]   inclusive state at the chunk's last token
+//   [0, 256)                       ticket counter (u32), zeroed before each launch
+//   agg  u64 [n][2(1+NS)][32]      aggregate map words, lane-minor
+//   incl u64 [n][2 NS][32]         inclusive-state words, lane-minor
+// Lane l of warp 0 owns channels 2l, 2l+1 of a chunk; word w of lane l holds
+// {epoch (high 32 bits), fp32 value (low 32 bits)}.  A 64-bit word is written
+// and read in one access, so a reader that sees the current launch's epoch
+// also sees its value: the descriptors need no flags, fences or reset, only
+// a zero fill before the workspace's first use (epoch 0 is never issued).
 struct Workspace {
   unsigned int* counter;
-  unsigned int* flags;
-  float* agg;
-  float* incl;
+  unsigned long long* agg;
+  unsigned long long* incl;
 };
 
 __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-constexpr int kFlagLanes = 32;   // lane l of warp 0 publishes channels 2l, 2l+1
+constexpr int kDescLanes = 32;
 
 inline size_t workspace_bytes(long long n_chunks, int NS) {
   size_t b = 256;
-  b += align256(sizeof(unsigned int) * kFlagLanes * n_chunks);
-  b += align256(sizeof(float) * n_chunks * (1 + NS) * kSlab);
-  b += align256(sizeof(float) * n_chunks * NS * kSlab);
+  b += align256(sizeof(unsigned long long) * n_chunks * 2 * (1 + NS) * kDescLanes);
+  b += align256(sizeof(unsigned long long) * n_chunks * 2 * NS * kDescLanes);
   return b;
 }
 
@@ -73,17 +75,31 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
   Workspace w;
   w.counter = reinterpret_cast<unsigned int*>(p);
   p += 256;
-  w.flags = reinterpret_cast<unsigned int*>(p);
-  p += align256(sizeof(unsigned int) * kFlagLanes * n_chunks);
-  w.agg = reinterpret_cast<float*>(p);
-  p += align256(sizeof(float) * n_chunks * (1 + NS) * kSlab);
-  w.incl = reinterpret_cast<float*>(p);
+  w.agg = reinterpret_cast<unsigned long long*>(p);
+  p += align256(sizeof(unsigned long long) * n_chunks * 2 * (1 + NS) * kDescLanes);
+  w.incl = reinterpret_cast<unsigned long long*>(p);
   return w;
 }
 
-// Bytes to zero before each launch: counter + flags.
-inline size_t reset_bytes(long long n_chunks) {
-  return 256 + align256(sizeof(unsigned int) * kFlagLanes * n_chunks);
+// Bytes to zero before each launch: the ticket counter.
+inline size_t reset_bytes(long long) { return 256; }
+
+__device__ __forceinline__ void put_word(unsigned long long* p, float v, unsigned int epoch) {
+  const unsigned long long w = ((unsigned long long)epoch << 32) | __float_as_uint(v);
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(w) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long get_word(const unsigned long long* p) {
+  unsigned long long w;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(w) : "l"(p) : "memory");
+  return w;
+}
+
+__device__ __forceinline__ bool word_ok(unsigned long long w, unsigned int epoch) {
+  return (unsigned int)(w >> 32) == epoch;
+}
+__device__ __forceinline__ float word_val(unsigned long long w) {
+  return __uint_as_float((unsigned int)w);
 }
 
 template <typename T, int NS>
@@ -91,6 +107,7 @@ struct Params {
   T* h[NS];
   float* final_state;     // nullable: [NS][B][C]
   Workspace ws;
+  unsigned int epoch;     // nonzero, unique per launch
   int B, Tn, C;           // Tn tokens, C = H * Dh channels per token
   int slabs;              // C / 64
   int n_chains;           // B * slabs
@@ -171,9 +188,8 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
       // publish a zero state so that successors do not wait on this chunk
       if (tid < 32) {
 #pragma unroll
-        for (int s = 0; s < NS; ++s)
-          __stcg(reinterpret_cast<float2*>(p.ws.incl + (desc * NS + s) * kSlab + 2 * tid), make_float2(0.f, 0.f));
-        st_release_gpu(p.ws.flags + desc * kFlagLanes + tid, 2u);
+        for (int w = 0; w < 2 * NS; ++w)
+          put_word(p.ws.incl + (desc * 2 * NS + w) * kDescLanes + tid, 0.f, p.epoch);
         if (tid == 0) raise_error(RATP_ERR_TIMEOUT);
       }
       return;
@@ -297,66 +313,65 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   }
 
   // ---- publish, look back, publish inclusive (warp 0) ----
-  // Lane l of warp 0 owns channels 2l, 2l+1 of the chunk descriptors: it
-  // writes them and then releases its own flag, and in a successor chunk the
-  // lane with the same index acquires that flag before reading them.  Every
-  // release/acquire pair is thread-to-thread, so no fence is needed.
+  // Lane l of warp 0 owns channels c0 = 2l, 2l+1: it writes its aggregate
+  // words, walks back over predecessor chunks of the chain reading the same
+  // lane's words (two predecessors per round trip), composing aggregates until
+  // it meets an inclusive state, then writes its own inclusive words.
   if (tid < 32) {
     const int lane = tid;
-    const unsigned int* cflags = p.ws.flags + (long long)chain * p.n_chunks_t * kFlagLanes + lane;
-    unsigned int* my_flag = p.ws.flags + desc * kFlagLanes + lane;
-    const float* agg = p.ws.agg;
-    float* incl = p.ws.incl;
+    constexpr int WA = 2 * (1 + NS), WI = 2 * NS;   // words per lane
+    const unsigned long long* agg = p.ws.agg;
+    const unsigned long long* incl = p.ws.incl;
+    const long long chain0 = (long long)chain * p.n_chunks_t;   // descriptor of chunk 0
     const int c0 = lane * 2;
     float cb0[NS], cb1[NS];
 #pragma unroll
     for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
-    if (chunk == 0) {
+    if (chunk > 0) {
+      unsigned long long* dst = p.ws.agg + desc * WA * kDescLanes + lane;
+      put_word(dst + 0 * kDescLanes, s_tot_a[c0], p.epoch);
+      put_word(dst + 1 * kDescLanes, s_tot_a[c0 + 1], p.epoch);
 #pragma unroll
-      for (int s = 0; s < NS; ++s)
-        __stcg(reinterpret_cast<float2*>(incl + (desc * NS + s) * kSlab + c0),
-               make_float2(s_tot_b[s][c0], s_tot_b[s][c0 + 1]));
-      st_release_gpu(my_flag, 2u);
-    } else {
-      {
-        float* dst = p.ws.agg + desc * (1 + NS) * kSlab;
-        __stcg(reinterpret_cast<float2*>(dst + c0), make_float2(s_tot_a[c0], s_tot_a[c0 + 1]));
-#pragma unroll
-        for (int s = 0; s < NS; ++s)
-          __stcg(reinterpret_cast<float2*>(dst + (1 + s) * kSlab + c0),
-                 make_float2(s_tot_b[s][c0], s_tot_b[s][c0 + 1]));
+      for (int s = 0; s < NS; ++s) {
+        put_word(dst + (2 + 2 * s) * kDescLanes, s_tot_b[s][c0], p.epoch);
+        put_word(dst + (3 + 2 * s) * kDescLanes, s_tot_b[s][c0 + 1], p.epoch);
       }
-      st_release_gpu(my_flag, 1u);
-
       // composite map of the predecessors composed so far: x -> ca x + cb
       float ca0 = 1.f, ca1 = 1.f;
       int top = chunk - 1;                      // nearest predecessor not yet composed
       const unsigned long long t_start = global_ns();
-      while (true) {
-        constexpr int kWin = 4;                 // predecessors polled at once
-        const int n = min(kWin, top + 1);
-        unsigned int f[kWin];
+      while (top >= 0) {
+        // words of predecessors top and top-1, all loads issued together
+        unsigned long long wi[2][WI], wa[2][WA];
 #pragma unroll
-        for (int u = 0; u < kWin; ++u) f[u] = (u < n) ? ld_acquire_gpu(cflags + (long long)(top - u) * kFlagLanes) : 0u;
-        int upto = -1;                          // aggregates to compose
-        bool found = false;                     // an inclusive state ends the walk
+        for (int u = 0; u < 2; ++u) {
+          const long long d = chain0 + (top - u);
+          const bool exists = (top - u) >= 0;
 #pragma unroll
-        for (int u = kWin - 1; u >= 0; --u) {   // nearest inclusive with no gap before it
-          if (u < n && f[u] >= 2u) { upto = u; found = true; }
+          for (int w = 0; w < WI; ++w) wi[u][w] = exists ? get_word(incl + (d * WI + w) * kDescLanes + lane) : 0ull;
+#pragma unroll
+          for (int w = 0; w < WA; ++w) wa[u][w] = exists ? get_word(agg + (d * WA + w) * kDescLanes + lane) : 0ull;
         }
-        if (found) {
+        bool inc[2], ag[2];
 #pragma unroll
-          for (int u = 0; u < kWin; ++u)
-            if (u < upto && f[u] == 0u) found = false;
-          if (!found) upto = -1;
-        } else {
-          bool all = true;
+        for (int u = 0; u < 2; ++u) {
+          inc[u] = true;
+          ag[u] = true;
 #pragma unroll
-          for (int u = 0; u < kWin; ++u)
-            if (u < n && f[u] == 0u) all = false;
-          if (all) upto = n;
+          for (int w = 0; w < WI; ++w) inc[u] = inc[u] && word_ok(wi[u][w], p.epoch);
+#pragma unroll
+          for (int w = 0; w < WA; ++w) ag[u] = ag[u] && word_ok(wa[u][w], p.epoch);
         }
-        if (upto < 0) {
+        // how far this round gets: compose n aggregates, then maybe an inclusive
+        int n = -1;
+        bool found = false;
+        if (inc[0]) { n = 0; found = true; }
+        else if (ag[0]) {
+          if (top >= 1 && inc[1]) { n = 1; found = true; }
+          else if (top >= 1 && ag[1]) n = 2;
+          else n = 1;
+        }
+        if (n < 0) {
           if (global_ns() - t_start > kSpinTimeoutNs) {
             raise_error(RATP_ERR_TIMEOUT);
             ca0 = ca1 = 0.f;                     // give up: zero carry
@@ -367,53 +382,39 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
           __nanosleep(20);
           continue;
         }
-        // all data loads of this window are issued before they are used
-        float2 pa[kWin], pb[NS][kWin], pv[NS];
 #pragma unroll
-        for (int u = 0; u < kWin; ++u) {
-          if (u < upto) {
-            const float* src = agg + ((long long)chain * p.n_chunks_t + (top - u)) * (1 + NS) * kSlab;
-            pa[u] = __ldcg(reinterpret_cast<const float2*>(src + c0));
-#pragma unroll
-            for (int s = 0; s < NS; ++s) pb[s][u] = __ldcg(reinterpret_cast<const float2*>(src + (1 + s) * kSlab + c0));
-          }
-        }
-        if (found) {
-          const long long dk = (long long)chain * p.n_chunks_t + (top - upto);
-#pragma unroll
-          for (int s = 0; s < NS; ++s) pv[s] = __ldcg(reinterpret_cast<const float2*>(incl + (dk * NS + s) * kSlab + c0));
-        }
-#pragma unroll
-        for (int u = 0; u < kWin; ++u) {
-          if (u < upto) {
+        for (int u = 0; u < 2; ++u) {
+          if (u < n) {
 #pragma unroll
             for (int s = 0; s < NS; ++s) {
-              cb0[s] = fmaf(ca0, pb[s][u].x, cb0[s]);
-              cb1[s] = fmaf(ca1, pb[s][u].y, cb1[s]);
+              cb0[s] = fmaf(ca0, word_val(wa[u][2 + 2 * s]), cb0[s]);
+              cb1[s] = fmaf(ca1, word_val(wa[u][3 + 2 * s]), cb1[s]);
             }
-            ca0 *= pa[u].x;
-            ca1 *= pa[u].y;
+            ca0 *= word_val(wa[u][0]);
+            ca1 *= word_val(wa[u][1]);
           }
         }
         if (found) {
 #pragma unroll
-          for (int s = 0; s < NS; ++s) {
-            cb0[s] = fmaf(ca0, pv[s].x, cb0[s]);   // carry = composite(inclusive)
-            cb1[s] = fmaf(ca1, pv[s].y, cb1[s]);
+          for (int s = 0; s < NS; ++s) {                           // carry = composite(inclusive)
+            const unsigned long long i0 = (n == 0) ? wi[0][2 * s] : wi[1][2 * s];
+            const unsigned long long i1 = (n == 0) ? wi[0][2 * s + 1] : wi[1][2 * s + 1];
+            cb0[s] = fmaf(ca0, word_val(i0), cb0[s]);
+            cb1[s] = fmaf(ca1, word_val(i1), cb1[s]);
           }
           break;
         }
-        top -= upto;
-        if (top < 0) break;                      // walked back to the sequence start
+        top -= n;
       }
-      // cb now holds the state entering this chunk; publish the inclusive state
+    }
+    // publish the inclusive state of this chunk
+    {
+      unsigned long long* dst = p.ws.incl + desc * (2 * NS) * kDescLanes + lane;
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        const float e0 = fmaf(s_tot_a[c0], cb0[s], s_tot_b[s][c0]);
-        const float e1 = fmaf(s_tot_a[c0 + 1], cb1[s], s_tot_b[s][c0 + 1]);
-        __stcg(reinterpret_cast<float2*>(incl + (desc * NS + s) * kSlab + c0), make_float2(e0, e1));
+        put_word(dst + (2 * s) * kDescLanes, fmaf(s_tot_a[c0], cb0[s], s_tot_b[s][c0]), p.epoch);
+        put_word(dst + (2 * s + 1) * kDescLanes, fmaf(s_tot_a[c0 + 1], cb1[s], s_tot_b[s][c0 + 1]), p.epoch);
       }
-      st_release_gpu(my_flag, 2u);
     }
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
