@@ -28,11 +28,14 @@
 //              pair exchanges the row max through shared memory, the running
 //              max is kept with O rescaled in TMEM only when it grows by more
 //              than 2^8, and P (bf16) is written into one of two 128B-swizzled
-//              K-major smem tiles; finally each thread normalises half an O row.
+//              K-major smem tiles.  An item's epilogue (normalise half an O
+//              row, store) runs after the softmax of the next item's first
+//              tile, so waiting for its last P V overlaps useful work.
 //   warp 8     TMA producer of Q and of a 2-stage K ring (a K stage is freed
 //              as soon as its S = Q K^T completes);
 //   warp 10    TMA producer of a 2-stage V ring (freed when P V completes);
-//   warp 9     allocates TMEM (512 columns: S ping-pong 2x128, O 128) and one
+//   warp 9     allocates TMEM (512 columns: S ping-pong 2x128, O ping-pong
+//              2x128, one O per work item in flight) and one
 //              lane issues S = Q K^T (SS, K-major) and O += P V (P K-major,
 //              V MN-major) as 128x128x16 tcgen05.mma; completions signal
 //              mbarriers via tcgen05.commit.
@@ -66,7 +69,7 @@ constexpr uint32_t kXchgBytes = 2 * BM * 4;                    // [2 halves][128
 constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + alignment slack
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;      // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;    // O at columns 256..383
+constexpr uint32_t kColO = 256;    // O double buffer at columns 256..383 and 384..511
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 struct Params {
@@ -235,9 +238,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       constexpr uint32_t idPV = idesc_bf16_f32(BM, DH, 0, 1);   // P V: V is MN-major
       int g = 0, li = 0;
       bool pend = false;
-      int pg = 0, pst = 0, pacc = 0;
+      int pg = 0, pst = 0, pacc = 0, pob = 0;
       bool ok = true;
-      auto issue_pv = [&](int gg, int stg, int acc) -> bool {
+      auto issue_pv = [&](int gg, int stg, int acc, int ob) -> bool {
         const int pb = gg & 1;
         if (!mbar_wait(b_pfull + 8 * pb, (gg >> 1) & 1, s_abort)) return false;
         if (!mbar_wait(b_vfull + 8 * stg, (gg / NST) & 1, s_abort)) return false;
@@ -246,7 +249,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         for (int k = 0; k < BN / 16; ++k) {
           const uint64_t a = sw128_desc(sP + pb * kTile + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
           const uint64_t bdesc = sw128_desc(sV + stg * kTile + k * 16 * 128, kHalf, 1024);
-          umma_f16(tmem + kColO, a, bdesc, idPV, (acc || k > 0) ? 1u : 0u);
+          umma_f16(tmem + kColO + ob * DH, a, bdesc, idPV, (acc || k > 0) ? 1u : 0u);
         }
         umma_commit(b_vempty + 8 * stg);
         umma_commit(b_pvdone + 8 * pb);
@@ -271,12 +274,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           umma_commit(b_sfull + 8 * sbuf);
           umma_commit(b_kempty + 8 * st);
           if (j == it.n_tiles - 1) umma_commit(b_qempty);
-          if (pend && !issue_pv(pg, pst, pacc)) { ok = false; break; }
+          if (pend && !issue_pv(pg, pst, pacc, pob)) { ok = false; break; }
           pend = true;
-          pg = g; pst = st; pacc = (j > 0);
+          pg = g; pst = st; pacc = (j > 0); pob = li & 1;
         }
       }
-      if (ok && pend) issue_pv(pg, pst, pacc);
+      if (ok && pend) issue_pv(pg, pst, pacc, pob);
     }
     __syncwarp();
   } else {
@@ -295,11 +298,46 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     // schedule early: after a failed (timed-out or aborted) wait the warps
     // carry on with whatever tensor memory holds; every later wait fails fast
     // and the error word already records the timeout.
-    int g = 0;
-    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+    // deferred epilogue of the previous item (-1: none): its item index, its
+    // O buffer, its last tile and this thread's partial row sum
+    int pend_idx = -1, pend_ob = 0, pend_gl = 0;
+    float pend_l = 0.f;
+    auto epilogue = [&](int e_idx, int e_ob, int e_gl, float e_l) {
+      const Item e = make_item(p, e_idx);
+      const int e_t = e.t0 + r;
+      warp_all(mbar_wait(b_pvdone + 8 * (e_gl & 1), (e_gl >> 1) & 1, s_abort));
+      tc_fence_after();
+      *x_mine = e_l;
+      pair_sync();
+      const float inv = 1.f / (e_l + *x_other);
+      pair_sync();
+      __nv_bfloat16* orow = p.o + (((size_t)e.b * p.T + e_t) * p.H + e.h) * DH + c_base;
+      const uint32_t ocol = kColO + e_ob * DH + c_base;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t o32[32];
+        tmem_ld32(tl + ocol + c * 32, o32);
+        tmem_wait_ld();
+        if (e_t < p.T) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 pk;
+            pk.x = pack_bf16x2(__uint_as_float(o32[8 * v + 0]) * inv, __uint_as_float(o32[8 * v + 1]) * inv);
+            pk.y = pack_bf16x2(__uint_as_float(o32[8 * v + 2]) * inv, __uint_as_float(o32[8 * v + 3]) * inv);
+            pk.z = pack_bf16x2(__uint_as_float(o32[8 * v + 4]) * inv, __uint_as_float(o32[8 * v + 5]) * inv);
+            pk.w = pack_bf16x2(__uint_as_float(o32[8 * v + 6]) * inv, __uint_as_float(o32[8 * v + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = pk;
+          }
+        }
+      }
+      tc_fence_before();
+    };
+    int g = 0, li = 0;
+    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x, ++li) {
       const Item it = make_item(p, idx);
+      const int ob = li & 1;
+      const uint32_t ocol_item = kColO + ob * DH + c_base;
       const int t = it.t0 + r;
-      const bool row_ok = t < p.T;
       const int lim_dil = it.dense ? (t + 1) : (t / it.Dd);
       const int w_lo = max(t - p.W_eff + 1, 0);
       float m_used = -1e30f, l = 0.f;
@@ -379,11 +417,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             uint32_t o32[32];
-            tmem_ld32(tl + kColO + c_base + c * 32, o32);
+            tmem_ld32(tl + ocol_item + c * 32, o32);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
-            tmem_st32(tl + kColO + c_base + c * 32, o32);
+            tmem_st32(tl + ocol_item + c * 32, o32);
           }
           tmem_wait_st();
           if (need) {
@@ -434,35 +472,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(b_pfull + 8 * sbuf);
-      }
-      // ---- epilogue: O / l -> bf16 -> global (each thread half a row)
-      const int gl = g - 1;
-      warp_all(mbar_wait(b_pvdone + 8 * (gl & 1), (gl >> 1) & 1, s_abort));
-      tc_fence_after();
-      *x_mine = l;
-      pair_sync();
-      const float inv = 1.f / (l + *x_other);
-      pair_sync();
-      __nv_bfloat16* orow = p.o + (((size_t)it.b * p.T + t) * p.H + it.h) * DH + c_base;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t o32[32];
-        tmem_ld32(tl + kColO + c_base + c * 32, o32);
-        tmem_wait_ld();
-        if (row_ok) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 pk;
-            pk.x = pack_bf16x2(__uint_as_float(o32[8 * v + 0]) * inv, __uint_as_float(o32[8 * v + 1]) * inv);
-            pk.y = pack_bf16x2(__uint_as_float(o32[8 * v + 2]) * inv, __uint_as_float(o32[8 * v + 3]) * inv);
-            pk.z = pack_bf16x2(__uint_as_float(o32[8 * v + 4]) * inv, __uint_as_float(o32[8 * v + 5]) * inv);
-            pk.w = pack_bf16x2(__uint_as_float(o32[8 * v + 6]) * inv, __uint_as_float(o32[8 * v + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = pk;
-          }
+        if (j == 0 && pend_idx >= 0) {
+          epilogue(pend_idx, pend_ob, pend_gl, pend_l);
+          pend_idx = -1;
         }
       }
-      tc_fence_before();
+      pend_idx = idx;
+      pend_ob = ob;
+      pend_gl = g - 1;
+      pend_l = l;
     }
+    if (pend_idx >= 0) epilogue(pend_idx, pend_ob, pend_gl, pend_l);
   }
 
   tc_fence_before();
