@@ -72,6 +72,24 @@ int ratp_last_error(void* stream);
 /* Number of SMs of the current device (grid sizing). */
 int ratp_device_sm_count(int* sms);
 
+/* Failure injection for tests of the error paths; never needed otherwise.
+ * Affects launches issued afterwards on the current device.
+ *   RATP_FAULT_NONE          restore the defaults (arg ignored);
+ *   RATP_FAULT_SPIN_LIMIT    bound, in ns, of every device-side wait
+ *                            (default 2e9); arg <= 0 restores the default;
+ *   RATP_FAULT_SCAN_DROP     the scan chunk with launch ticket `arg` publishes
+ *                            no descriptor, so its successor's wait runs out;
+ *   RATP_FAULT_ATTN_DROP_K   the first CTA of the tensor-core attention never
+ *                            loads its K tile number `arg`, so the MMA's wait
+ *                            runs out.
+ * A wait that runs out ends its kernel early with RATP_ERR_TIMEOUT in the
+ * device error word (outputs are then undefined); the context stays usable.
+ * Returns RATP_ERR_ARG for an unknown kind, RATP_ERR_CUDA if the device
+ * update fails.  Not thread-safe with concurrent launches. */
+enum { RATP_FAULT_NONE = 0, RATP_FAULT_SPIN_LIMIT = 1, RATP_FAULT_SCAN_DROP = 2,
+       RATP_FAULT_ATTN_DROP_K = 3 };
+int ratp_debug_fault(int kind, long long arg);
+
 /* ------------------------------------------------------------------------
  * Prefill recurrence (write-up section 2.1).
  *

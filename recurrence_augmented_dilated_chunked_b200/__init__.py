@@ -12,11 +12,13 @@ from ._binding import (  # noqa: F401
     RatpError,
     dilated_attn_prefill,
     dilated_attn_prefill_simt,
+    debug_fault,
     exported_symbols,
     last_error,
     load_library,
     scan_prefill,
     scan_prefill_kv,
+    scan_prefill_kv_noalloc,
     scan_workspace,
     sm_count,
 )

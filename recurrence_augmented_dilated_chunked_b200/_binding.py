@@ -51,6 +51,7 @@ _SIGS = {
     "ratp_status_string": ([_I], ctypes.c_char_p),
     "ratp_last_error": ([_P], _I),
     "ratp_device_sm_count": ([ctypes.POINTER(_I)], _I),
+    "ratp_debug_fault": ([_I, ctypes.c_longlong], _I),
     "ratp_scan_workspace_bytes": ([_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "ratp_scan_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "ratp_scan_prefill_kv": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
@@ -224,6 +225,14 @@ def last_error(device=None):
     dev = torch.device("cuda" if device is None else device)
     s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     _check("ratp_last_error", lib.ratp_last_error(s))
+
+
+FAULT_NONE, FAULT_SPIN_LIMIT, FAULT_SCAN_DROP, FAULT_ATTN_DROP_K = 0, 1, 2, 3
+
+
+def debug_fault(kind: int, arg: int = 0):
+    """Plant a failure for tests of the error paths (see ``ratp_debug_fault``)."""
+    _check("ratp_debug_fault", load_library().ratp_debug_fault(int(kind), int(arg)))
 
 
 def sm_count() -> int:

@@ -224,6 +224,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             if (it.dense) m = is_k ? &tm_kpos : &tm_vpos;
             else m = is_k ? &tm_kdil : &tm_vdil;
           }
+          if (is_k && blockIdx.x == 0 && (long long)g == g_fault_attn_ktile) continue;   // planted failure
           const uint32_t fb = b_full + 8 * st;
           mbar_arrive_expect_tx(fb, kTile);
           tma_load_4d(ring + st * kTile, m, fb, 0, it.h, row, it.b);

@@ -17,8 +17,14 @@ __device__ __forceinline__ void raise_error(unsigned int code) {
 }
 
 // Bound for every spin-wait (ns of %globaltimer).  A wait that runs out sets
-// RATP_ERR_TIMEOUT and the kernel carries on to a clean exit.
+// RATP_ERR_TIMEOUT and the kernel carries on to a clean exit.  Tests of the
+// failure paths lower it and plant a missing publication (ratp_debug_fault).
 constexpr unsigned long long kSpinTimeoutNs = 2000000000ull;
+__device__ unsigned long long g_spin_timeout_ns = kSpinTimeoutNs;
+__device__ long long g_fault_scan_ticket = -1;    // scan chunk that publishes nothing
+__device__ long long g_fault_attn_ktile = -1;     // K tile the first attention CTA skips
+
+__device__ __forceinline__ unsigned long long spin_timeout() { return g_spin_timeout_ns; }
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;

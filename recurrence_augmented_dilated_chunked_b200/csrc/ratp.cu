@@ -136,7 +136,9 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   if (!ensure_smem(scan::scan_kernel<T, NS>, smem)) return RATP_ERR_CUDA;
   cudaError_t e = cudaMemsetAsync(ws, 0, scan::reset_bytes(geo.n_chunks), st);
   if (e != cudaSuccess) return RATP_ERR_CUDA;
-  scan::scan_kernel<T, NS><<<(unsigned)geo.n_chunks, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);
+  // persistent: two CTAs per SM (the pipeline holds two chunks per CTA)
+  const long long grid = geo.n_chunks < 2LL * sm_count() ? geo.n_chunks : 2LL * sm_count();
+  scan::scan_kernel<T, NS><<<(unsigned)grid, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);
   return launch_status();
 }
 
@@ -392,6 +394,34 @@ int ratp_last_error(void* stream) {
   if (cudaMemcpyToSymbol(ratp::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return RATP_ERR_CUDA;
   for (int code = 1; code < 32; ++code)
     if (word & (1u << code)) return code;
+  return RATP_OK;
+}
+
+int ratp_debug_fault(int kind, long long arg) {
+  unsigned long long timeout = ratp::kSpinTimeoutNs;
+  long long scan = -1, attn = -1;
+  switch (kind) {
+    case RATP_FAULT_NONE: break;
+    case RATP_FAULT_SPIN_LIMIT: if (arg > 0) timeout = (unsigned long long)arg; break;
+    case RATP_FAULT_SCAN_DROP: scan = arg; break;
+    case RATP_FAULT_ATTN_DROP_K: attn = arg; break;
+    default: return RATP_ERR_ARG;
+  }
+  // a drop keeps the current wait bound; a new bound keeps the drops
+  if (kind == RATP_FAULT_SCAN_DROP || kind == RATP_FAULT_ATTN_DROP_K) {
+    if (cudaMemcpyFromSymbol(&timeout, ratp::g_spin_timeout_ns, sizeof(timeout)) != cudaSuccess) return RATP_ERR_CUDA;
+    long long other = -1;
+    if (cudaMemcpyFromSymbol(&other, kind == RATP_FAULT_SCAN_DROP ? ratp::g_fault_attn_ktile : ratp::g_fault_scan_ticket,
+                             sizeof(other)) != cudaSuccess) return RATP_ERR_CUDA;
+    if (kind == RATP_FAULT_SCAN_DROP) attn = other; else scan = other;
+  } else if (kind == RATP_FAULT_SPIN_LIMIT) {
+    if (cudaMemcpyFromSymbol(&scan, ratp::g_fault_scan_ticket, sizeof(scan)) != cudaSuccess ||
+        cudaMemcpyFromSymbol(&attn, ratp::g_fault_attn_ktile, sizeof(attn)) != cudaSuccess) return RATP_ERR_CUDA;
+  }
+  if (cudaMemcpyToSymbol(ratp::g_spin_timeout_ns, &timeout, sizeof(timeout)) != cudaSuccess ||
+      cudaMemcpyToSymbol(ratp::g_fault_scan_ticket, &scan, sizeof(scan)) != cudaSuccess ||
+      cudaMemcpyToSymbol(ratp::g_fault_attn_ktile, &attn, sizeof(attn)) != cudaSuccess)
+    return RATP_ERR_CUDA;
   return RATP_OK;
 }
 

@@ -23,7 +23,7 @@
 //     and composes their aggregates until it meets an inclusive state.  The chunk stays
 //     in shared memory (TMA-filled) while it waits, so x and g are read from
 //     HBM exactly once.
-//   * every wait is bounded (kSpinTimeoutNs); on expiry the kernel records
+//   * every wait is bounded (spin_timeout()); on expiry the kernel records
 //     RATP_ERR_TIMEOUT and finishes with a zero carry.
 #pragma once
 #include "common.cuh"
@@ -45,7 +45,8 @@ struct Shape {
 };
 
 // Workspace layout (bytes), given n = total chunks and NS streams:
-//   [0, 256)                       ticket counter (u32), zeroed before each launch
+//   [0, 256)                       ticket counter (u32) and abort word (u32 at
+//                                  byte 128), zeroed before each launch
 //   agg  u64 [n][2(1+NS)][32]      aggregate map words, lane-minor
 //   incl u64 [n][2 NS][32]         inclusive-state words, lane-minor
 // Lane l of warp 0 owns channels 2l, 2l+1 of a chunk; word w of lane l holds
@@ -55,6 +56,7 @@ struct Shape {
 // a zero fill before the workspace's first use (epoch 0 is never issued).
 struct Workspace {
   unsigned int* counter;
+  unsigned int* abort;
   unsigned long long* agg;
   unsigned long long* incl;
 };
@@ -74,6 +76,7 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
   char* p = static_cast<char*>(base);
   Workspace w;
   w.counter = reinterpret_cast<unsigned int*>(p);
+  w.abort = reinterpret_cast<unsigned int*>(p + 128);
   p += 256;
   w.agg = reinterpret_cast<unsigned long long*>(p);
   p += align256(sizeof(unsigned long long) * n_chunks * 2 * (1 + NS) * kDescLanes);
@@ -122,11 +125,12 @@ struct Smem {
   static constexpr int kData = (1 + NS) * kTile;
   // per-warp totals of the intra-chunk scan: [warps][1 + NS][kSlab] floats
   static constexpr int kScan = (kThreads / 32) * (1 + NS) * kSlab * 4;
-  static constexpr int kBytes = kData + kScan + 128;                       // + alignment
+  static constexpr int kStages = 2;                                        // chunk pipeline depth
+  static constexpr int kBytes = kStages * kData + kScan + 128;             // + alignment
 };
 
 template <typename T, int NS>
-__global__ void __launch_bounds__(kThreads, 4)
+__global__ void __launch_bounds__(kThreads, 2)
 scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x0,
             const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ Params<T, NS> p) {
   using S = Shape<T>;
@@ -135,39 +139,61 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  const T* s_g = reinterpret_cast<const T*>(smem);
   constexpr int NW = kThreads / 32;
-  float* s_w = reinterpret_cast<float*>(smem + SM::kData);            // [NW][1 + NS][64]
-  __shared__ __align__(8) uint64_t s_bar;
-  __shared__ unsigned int s_ticket;
+  constexpr int NSTG = SM::kStages;
+  float* s_w = reinterpret_cast<float*>(smem + NSTG * SM::kData);    // [NW][1 + NS][64]
+  __shared__ __align__(8) uint64_t s_bar[NSTG];
+  __shared__ unsigned int s_ticket[NSTG];
   __shared__ float s_tot_a[kSlab];
   __shared__ float s_tot_b[NS][kSlab];
   __shared__ float s_carry[NS][kSlab];
   static_assert(32 % LANES == 0, "row groups of a warp must share channels");
 
   const int tid = threadIdx.x;
-  const uint32_t bar = sm100::smem_u32(&s_bar);
+  const unsigned int n_total = (unsigned int)p.n_chains * (unsigned int)p.n_chunks_t;
+  // TMA loads of chunk `tk` (gate tile first) into pipeline stage `stg`;
+  // rows past T read as zero
+  auto fetch = [&](unsigned int tk, int stg) {
+    const int ck = tk / p.n_chains, chn = tk % p.n_chains;
+    const uint32_t bb = sm100::smem_u32(&s_bar[stg]);
+    sm100::mbar_arrive_expect_tx(bb, SM::kData);
+    const uint32_t dst = sm100::smem_u32(smem + stg * SM::kData);
+    const int x = (chn % p.slabs) * kSlab, y = ck * L, z = chn / p.slabs;
+    sm100::tma_load_3d(dst, &tm_g, bb, x, y, z);
+    sm100::tma_load_3d(dst + SM::kTile, &tm_x0, bb, x, y, z);
+    if (NS == 2) sm100::tma_load_3d(dst + 2 * SM::kTile, &tm_x1, bb, x, y, z);
+  };
+  auto aborted = [&]() -> bool {
+    unsigned int v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.ws.abort) : "memory");
+    return v != 0u;
+  };
   if (tid == 0) {
-    s_ticket = atomicAdd(p.ws.counter, 1u);
-    sm100::mbar_init(bar, 1);
+    for (int i = 0; i < NSTG; ++i) sm100::mbar_init(sm100::smem_u32(&s_bar[i]), 1);
     sm100::fence_barrier_init();
+    const unsigned int tk = atomicAdd(p.ws.counter, 1u);
+    s_ticket[0] = tk;
+    if (tk < n_total) fetch(tk, 0);
   }
   __syncthreads();
-  const unsigned int ticket = s_ticket;
-  const int chunk = ticket / p.n_chains;     // chunk-major: predecessors started earlier
+
+  // Persistent loop: chunk tickets come in launch order; while this CTA scans
+  // one chunk, the next ticket's tiles are already being loaded.
+  for (int it = 0;; ++it) {
+  const int stage = it & 1;
+  const unsigned int ticket = s_ticket[stage];
+  if (ticket >= n_total) break;
+  if (tid == 0) {
+    const unsigned int nx = atomicAdd(p.ws.counter, 1u);
+    s_ticket[stage ^ 1] = nx;
+    if (nx < n_total) fetch(nx, stage ^ 1);
+  }
+  const T* s_g = reinterpret_cast<const T*>(smem + stage * SM::kData);
+  const int chunk = ticket / p.n_chains;     // chunk-major: predecessors were ticketed earlier
   const int chain = ticket % p.n_chains;
   const int b = chain / p.slabs;
   const int slab = chain % p.slabs;
   const long long desc = (long long)chain * p.n_chunks_t + chunk;   // descriptor index
-
-  // ---- TMA: gate and input tiles of this chunk (rows past T read as zero) ----
-  if (tid == 0) {
-    sm100::mbar_arrive_expect_tx(bar, SM::kData);
-    const uint32_t dst = sm100::smem_u32(smem);
-    sm100::tma_load_3d(dst, &tm_g, bar, slab * kSlab, chunk * L, b);
-    sm100::tma_load_3d(dst + SM::kTile, &tm_x0, bar, slab * kSlab, chunk * L, b);
-    if (NS == 2) sm100::tma_load_3d(dst + 2 * SM::kTile, &tm_x1, bar, slab * kSlab, chunk * L, b);
-  }
 
   const int lane_c = tid % LANES;            // 16-byte column within the slab
   const int grp = tid / LANES;               // row group
@@ -178,21 +204,41 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   const int soff = grp * kRows * kSlab + lane_c * V;   // element offset of row 0 in a tile
 
   {
-    // bounded wait for the tiles (uniform outcome across the CTA)
-    const unsigned long long tw = global_ns();
+    // one thread waits for the tiles (bounded; the clock and the abort word
+    // are read every 64 polls), the others sleep in the barrier
     bool ok = true;
-    while (!sm100::mbar_try_wait(bar, 0)) {
-      if (global_ns() - tw > kSpinTimeoutNs) { ok = false; break; }
+    if (tid == 0) {
+      const uint32_t bb = sm100::smem_u32(&s_bar[stage]);
+      unsigned long long tw = 0;
+      unsigned int n = 0;
+      while (!sm100::mbar_try_wait(bb, (it >> 1) & 1)) {
+        if ((++n & 63u) == 0u) {
+          const unsigned long long now = global_ns();
+          if (tw == 0) tw = now;
+          else if (now - tw > spin_timeout() || aborted()) { ok = false; break; }
+        }
+      }
     }
     if (!__syncthreads_and(ok)) {
-      // publish a zero state so that successors do not wait on this chunk
+      // give up: publish a zero state for this chunk, make every other CTA
+      // stop waiting, and leave
       if (tid < 32) {
 #pragma unroll
         for (int w = 0; w < 2 * NS; ++w)
           put_word(p.ws.incl + (desc * 2 * NS + w) * kDescLanes + tid, 0.f, p.epoch);
-        if (tid == 0) raise_error(RATP_ERR_TIMEOUT);
+        if (tid == 0) {
+          raise_error(RATP_ERR_TIMEOUT);
+          atomicExch(p.ws.abort, 1u);
+          // let the prefetch into the other stage land before the CTA exits
+          if (s_ticket[stage ^ 1] < n_total) {
+            const uint32_t bo = sm100::smem_u32(&s_bar[stage ^ 1]);
+            const unsigned long long t1 = global_ns();
+            while (!sm100::mbar_try_wait(bo, ((it + 1) >> 1) & 1) && global_ns() - t1 < spin_timeout()) {
+            }
+          }
+        }
       }
-      return;
+      break;
     }
   }
 
@@ -319,6 +365,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   // it meets an inclusive state, then writes its own inclusive words.
   if (tid < 32) {
     const int lane = tid;
+    const bool drop = (long long)ticket == g_fault_scan_ticket;   // planted failure: publish nothing
     constexpr int WA = 2 * (1 + NS), WI = 2 * NS;   // words per lane
     const unsigned long long* agg = p.ws.agg;
     const unsigned long long* incl = p.ws.incl;
@@ -327,7 +374,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     float cb0[NS], cb1[NS];
 #pragma unroll
     for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
-    if (chunk > 0) {
+    if (chunk > 0 && !drop) {
       unsigned long long* dst = p.ws.agg + desc * WA * kDescLanes + lane;
       put_word(dst + 0 * kDescLanes, s_tot_a[c0], p.epoch);
       put_word(dst + 1 * kDescLanes, s_tot_a[c0 + 1], p.epoch);
@@ -336,6 +383,8 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
         put_word(dst + (2 + 2 * s) * kDescLanes, s_tot_b[s][c0], p.epoch);
         put_word(dst + (3 + 2 * s) * kDescLanes, s_tot_b[s][c0 + 1], p.epoch);
       }
+    }
+    if (chunk > 0) {
       // composite map of the predecessors composed so far: x -> ca x + cb
       float ca0 = 1.f, ca1 = 1.f;
       int top = chunk - 1;                      // nearest predecessor not yet composed
@@ -372,8 +421,9 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
           else n = 1;
         }
         if (n < 0) {
-          if (global_ns() - t_start > kSpinTimeoutNs) {
+          if (global_ns() - t_start > spin_timeout() || aborted()) {
             raise_error(RATP_ERR_TIMEOUT);
+            atomicExch(p.ws.abort, 1u);
             ca0 = ca1 = 0.f;                     // give up: zero carry
 #pragma unroll
             for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
@@ -408,7 +458,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
       }
     }
     // publish the inclusive state of this chunk
-    {
+    if (!drop) {
       unsigned long long* dst = p.ws.incl + desc * (2 * NS) * kDescLanes + lane;
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
@@ -453,6 +503,8 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
         }
       }
     }
+  }
+  __syncthreads();   // stage and ticket slot may be refilled from here on
   }
 }
 

@@ -43,7 +43,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity.  Returns false (and
-// records RATP_ERR_TIMEOUT) if it has not completed within kSpinTimeoutNs or
+// records RATP_ERR_TIMEOUT) if it has not completed within spin_timeout() or
 // if *abort is set by another role.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -53,7 +53,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0u) {
       if (*abort) return false;
-      if (global_ns() - t0 > kSpinTimeoutNs) {
+      if (global_ns() - t0 > spin_timeout()) {
         *abort = 1;
         raise_error(RATP_ERR_TIMEOUT);
         return false;

@@ -52,6 +52,11 @@ def test_cache_struct_matches_header():
     assert _struct_fields(body) == [f[0] for f in _binding.CacheStruct._fields_]
 
 
+def test_debug_fault_rejects_unknown_kind_on_host(lib):
+    assert lib.ratp_debug_fault(99, 0) == 1
+    assert lib.ratp_debug_fault(-1, 0) == 1
+
+
 def test_status_strings(lib):
     assert lib.ratp_status_string(0) == b"ok"
     assert b"aligned" in lib.ratp_status_string(3)
