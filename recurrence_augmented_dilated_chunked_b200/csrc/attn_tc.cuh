@@ -14,10 +14,12 @@
 //     gather is an ordinary box of the strided tensor map; a dense head reads
 //     the positional view instead (slot = position);
 //   * window tiles (dilated heads only): positions of [t0 - W' + 1, t_last],
-//     W' = max(W, 1), so W = 0 still supplies the self key t; window keys that
-//     are also dilated keys (j mod D = D-1, j < t) are masked out.
-// Per-row validity is a prefix (dilated: s < floor(t / D_h), dense: s <= t) or
-// a range minus a periodic pattern (window), evaluated in registers.
+//     W' = max(W, 1), so W = 0 still supplies the self key t.
+// Each key is counted once by splitting the set at the window: row t takes
+// every window position t-W'+1..t and only the dilated slots whose position
+// lies before the window, s < floor((t - W' + 1) / D).  So per-row validity is
+// a prefix (dilated; dense: s <= t) or a contiguous range (window), evaluated
+// as bit masks per 32-column chunk.
 //
 // Roles (352 threads, one CTA per SM, persistent over items in heavy-first
 // order -- dense heads and late query tiles first, round-robin over CTAs):
@@ -115,7 +117,7 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
     it.n_tiles = (it.t_last + 1 + BN - 1) / BN;
   } else {
     it.Dd = p.D;
-    const int n_dil = it.t_last / p.D;
+    const int n_dil = max(0, it.t_last - p.W_eff + 1) / p.D;   // slots before the last row's window
     it.p_start = max(0, it.t0 - p.W_eff + 1);
     it.n_win = (it.t_last - it.p_start + 1 + BN - 1) / BN;
     it.n_tiles = it.n_win + (n_dil + BN - 1) / BN;
@@ -339,7 +341,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int ob = li & 1;
       const uint32_t ocol_item = kColO + ob * DH + c_base;
       const int t = it.t0 + r;
-      const int lim_dil = it.dense ? (t + 1) : (t / it.Dd);
+      const int lim_dil = it.dense ? (t + 1) : (max(0, t - p.W_eff + 1) / it.Dd);
       const int w_lo = max(t - p.W_eff + 1, 0);
       float m_used = -1e30f, l = 0.f;
       for (int j = 0; j < it.n_tiles; ++j, ++g) {
@@ -355,27 +357,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 
         // validity bit masks of the two 32-column chunks of this half
         uint32_t vm[2];
-        if (j < it.n_win) {
-          const int p0 = it.p_start + j * BN + c_base;       // position of column 0 of the half
+        {
+          const int lim_lo = (j < it.n_win) ? (w_lo - (it.p_start + j * BN) - c_base) : 0;
+          const int lim_hi = (j < it.n_win) ? (t - (it.p_start + j * BN) - c_base + 1)
+                                            : (lim_dil - (j - it.n_win) * BN - c_base);
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
-            const int cb = p0 + 32 * k;
-            const int lo = min(max(w_lo - cb, 0), 32);         // first valid bit
-            const int hi = min(max(t - cb + 1, 0), 32);        // one past the last valid bit
-            uint32_t m = (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~(lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u));
-            // keys already in the dilated set: positions q = D-1 (mod D), q < t
-            const int lim = min(max(t - cb, 0), 32);
-            int i0 = (it.Dd - 1) - (cb % it.Dd);
-            if (i0 < 0) i0 += it.Dd;
-            for (int i = i0; i < lim; i += it.Dd) m &= ~(1u << i);
-            vm[k] = m;
-          }
-        } else {
-          const int lim = lim_dil - (j - it.n_win) * BN - c_base;
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int n = min(max(lim - 32 * k, 0), 32);
-            vm[k] = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+            const int lo = min(max(lim_lo - 32 * k, 0), 32);   // first valid column of the chunk
+            const int hi = min(max(lim_hi - 32 * k, 0), 32);   // one past the last valid column
+            vm[k] = (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~(lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u));
           }
         }
         // masked row max of this half (raw scores)

@@ -5,9 +5,9 @@
 //
 // Decode step for token t = len[b] of every sequence, one launch:
 //   grid (split, h, b).  The keys of (b, h) form a virtual list: the cached
-//   dilated slots s < t / D_h (Kc/Vc rows), then the raw window positions
-//   t-W < p < t (ring rows; positions with p mod D_h = D_h-1 are dilated keys
-//   already in the list and are skipped).  Split i streams keys
+//   dilated slots whose positions lie before the window, s < (t-W+1) / D_h
+//   (all s < t / D_h without a window; Kc/Vc rows), then every window position
+//   t-W < p < t (ring rows), so each key appears once.  Split i streams keys
 //   [i*split_keys, (i+1)*split_keys) with 16-byte loads, a half-warp per key
 //   (Dh = 128) and an fp32 online softmax per half-warp.
 //   Split 0 additionally performs the recurrence step for the k and v streams
@@ -78,15 +78,17 @@ decode_kernel(const Params p) {
   const bool dense = is_dense(p.dense_bits, h);
   const int Dd = dense ? 1 : p.D;
   bool active = true;
-  int n_slots = 0, w_lo = 0, n_win = 0, n_keys = 0, n_used = 1;
+  int n_slots = 0, w_lo = 0, n_win = 0, n_keys = 0, n_used = 1, app_slot = 0;
   if (t >= p.T_max) {
     active = false;
     if (split == 0 && h == 0 && tid == 0) raise_error(RATP_ERR_CAPACITY);
   } else {
-    n_slots = t / Dd;
+    app_slot = t / Dd;                           // slot of position t if it is a dilated one
+    n_slots = app_slot;
     if (p.W > 0 && !dense) {
       w_lo = max(0, t - p.W + 1);
       n_win = t - w_lo;
+      n_slots = w_lo / Dd;                       // dilated slots before the window
     }
     n_keys = n_slots + n_win;
     n_used = max(1, (n_keys + p.split_keys - 1) / p.split_keys);
@@ -109,12 +111,12 @@ decode_kernel(const Params p) {
         *st = hn;
         const __nv_bfloat16 hb = __float2bfloat16_rn(hn);
         (s == 0 ? s_self_k : s_self_v)[ch] = __bfloat162float(hb);
-        if (t % Dd == Dd - 1 && n_slots < p.T_max / Dd)
-          (s == 0 ? p.Kc : p.Vc)[(cache_row0 + n_slots) * DH + ch] = hb;
+        if (t % Dd == Dd - 1 && app_slot < p.T_max / Dd)
+          (s == 0 ? p.Kc : p.Vc)[(cache_row0 + app_slot) * DH + ch] = hb;
         if (p.W > 0)
           (s == 0 ? p.Kw : p.Vw)[(bh * p.W + t % p.W) * DH + ch] = hb;
       }
-      if (t % Dd == Dd - 1 && n_slots >= p.T_max / Dd && tid == 0) raise_error(RATP_ERR_CAPACITY);
+      if (t % Dd == Dd - 1 && app_slot >= p.T_max / Dd && tid == 0) raise_error(RATP_ERR_CAPACITY);
       __syncthreads();
     }
 
@@ -154,7 +156,7 @@ decode_kernel(const Params p) {
             const long long rr = (bh * p.W + pos % p.W) * DH;
             kr = p.Kw + rr;
             vr = p.Vw + rr;
-            use[u] = (pos % Dd) != (Dd - 1);
+            use[u] = true;
           }
           if (use[u]) {
             kv[u] = __ldcs(reinterpret_cast<const uint4*>(kr + li * 8));

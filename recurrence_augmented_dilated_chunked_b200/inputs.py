@@ -94,7 +94,8 @@ def decode_inputs(steps, B, H, Dh, dtype="bf16", gate_mean=2.0, gate_std=1.0, se
 
 def decode_context(B, H, Dh, ctx, D, W, dense_mask=None, seed=2):
     """Synthetic already-prefilled decode context: every cached dilated row,
-    every window-ring row and the fp32 recurrent state drawn from N(0, 1).
+    every window-ring row and the fp32 recurrent state drawn from N(0, 1); a
+    position held both as a dilated row and in the ring gets the one value.
 
     Returns (kd, vd, kw, vw, state): kd/vd are lists over heads of
     [B, ctx // D_h, Dh] bf16 tensors (row s = position s*D_h + D_h - 1);
@@ -112,4 +113,13 @@ def decode_context(B, H, Dh, ctx, D, W, dense_mask=None, seed=2):
     kw = torch.randn((B, H, Wr, Dh), generator=gen).to(torch.bfloat16)
     vw = torch.randn((B, H, Wr, Dh), generator=gen).to(torch.bfloat16)
     state = torch.randn((2, B, H, Dh), generator=gen, dtype=torch.float32)
+    # a position kept in both places (a dilated one inside the last W) holds
+    # one value, as it would after a prefill: the ring row repeats the slot
+    if W > 0:
+        for h in range(H):
+            Dd = 1 if (dense_mask is not None and dense_mask[h]) else D
+            for pos in range(max(0, ctx - W), ctx):
+                if pos % Dd == Dd - 1:
+                    kw[:, h, pos % W] = kd[h][:, pos // Dd]
+                    vw[:, h, pos % W] = vd[h][:, pos // Dd]
     return kd, vd, kw, vw, state
