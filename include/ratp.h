@@ -133,8 +133,9 @@ int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
  * ratp_scan_prefill_kv (the caller still provides and owns all tensors), and
  * the call itself performs no allocation of any kind.
  *   - A shape whose scratch would not fit returns RATP_ERR_CAPACITY
- *     (bf16: at most ~11,900 chunks of 128 tokens x 64 channels, i.e.
- *     B*T*H*Dh up to ~97 million elements; fp32 chunks hold 64 tokens).
+ *     (at most 6,553 chunks of 64 channels x 256 tokens for bf16, i.e.
+ *     B*T*H*Dh up to ~107 million elements; fp32 chunks hold 128 tokens,
+ *     ~53 million elements).
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
  *   - All calls share the one array, which keeps the previous call's

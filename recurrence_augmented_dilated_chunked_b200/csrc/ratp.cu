@@ -136,9 +136,8 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   if (!ensure_smem(scan::scan_kernel<T, NS>, smem)) return RATP_ERR_CUDA;
   cudaError_t e = cudaMemsetAsync(ws, 0, scan::reset_bytes(geo.n_chunks), st);
   if (e != cudaSuccess) return RATP_ERR_CUDA;
-  // persistent: two CTAs per SM (the pipeline holds two chunks per CTA)
-  const long long grid = geo.n_chunks < 2LL * sm_count() ? geo.n_chunks : 2LL * sm_count();
-  scan::scan_kernel<T, NS><<<(unsigned)grid, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);
+  // one CTA per chunk; chunk tickets, not block indices, fix the order
+  scan::scan_kernel<T, NS><<<(unsigned)geo.n_chunks, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);
   return launch_status();
 }
 

@@ -8,23 +8,23 @@
 //
 // Decomposition (B200-first, HBM bound):
 //   * a "chain" is one batch item x one slab of 64 contiguous channels; a
-//     chunk is L consecutive tokens of one chain (L = 128 for bf16, 64 for
-//     fp32).  One CTA of 256 threads owns one chunk.  Lanes cover contiguous
-//     channels with 16-byte vectors, so every load instruction of a warp reads
-//     whole 128-byte lines; each thread holds R = 4 consecutive tokens.
-//   * in registers: each thread reduces its 4 tokens to one affine map; the
-//     row groups of a warp are combined by a shuffle scan, the 8 warp totals
-//     by one warp through shared memory.
+//     chunk is L consecutive tokens of one chain.  One CTA of 256 threads owns
+//     one chunk, staged by TMA into shared memory (gate tile + one tile per
+//     stream).  A thread holds R consecutive tokens x 8 (bf16; 4 for fp32)
+//     contiguous channels, works on channel pairs with packed f32x2
+//     arithmetic, and reduces its tokens to one affine map per channel.
+//   * within the chunk: the row groups of a warp are combined by a shuffle
+//     scan, the 8 warp totals by one warp through shared memory.
 //   * across chunks: decoupled look-back.  Chunk tickets come from an atomic
 //     counter in launch order, so a CTA only waits on chunks whose CTAs have
 //     started.  Each lane of warp 0 owns two channels of the chunk's
 //     descriptor: it publishes its part of the aggregate map at once as
 //     epoch-tagged 64-bit words, then reads two predecessors per round trip
-//     and composes their aggregates until it meets an inclusive state.  The chunk stays
-//     in shared memory (TMA-filled) while it waits, so x and g are read from
-//     HBM exactly once.
+//     and composes their aggregates until it meets an inclusive state.  x and
+//     g are read from HBM exactly once.
 //   * every wait is bounded (spin_timeout()); on expiry the kernel records
-//     RATP_ERR_TIMEOUT and finishes with a zero carry.
+//     RATP_ERR_TIMEOUT, sets a kernel-wide abort word so that no other CTA
+//     keeps waiting, and finishes with a zero carry.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -34,14 +34,17 @@ namespace scan {
 
 constexpr int kThreads = 256;
 constexpr int kSlab = 64;   // channels per chain
-constexpr int kRows = 4;    // tokens per thread
+#ifndef RATP_SCAN_ROWS
+#define RATP_SCAN_ROWS 8
+#endif
+constexpr int kRows = RATP_SCAN_ROWS;   // tokens per thread
 
-template <typename T>
+template <typename T, int R = kRows>
 struct Shape {
   static constexpr int kVec = Elem<T>::kVec;             // channels per 16 B
   static constexpr int kLanes = kSlab / kVec;            // threads per token row
   static constexpr int kGroups = kThreads / kLanes;      // row groups per CTA
-  static constexpr int kChunk = kGroups * kRows;         // tokens per chunk
+  static constexpr int kChunk = kGroups * R;             // tokens per chunk
 };
 
 // Workspace layout (bytes), given n = total chunks and NS streams:
@@ -118,100 +121,80 @@ struct Params {
 };
 
 // Dynamic shared memory: (1 + NS) tiles of [chunk][64] elements filled by TMA
-// (the gate tile first), then the row-group maps of the intra-chunk scan.
-template <typename T, int NS>
+// (the gate tile first), then the per-warp totals of the intra-chunk scan.
+template <typename T, int NS, int R = kRows>
 struct Smem {
-  static constexpr int kTile = Shape<T>::kChunk * kSlab * (int)sizeof(T);   // 16 KB
+  static constexpr int kTile = Shape<T, R>::kChunk * kSlab * (int)sizeof(T);
   static constexpr int kData = (1 + NS) * kTile;
-  // per-warp totals of the intra-chunk scan: [warps][1 + NS][kSlab] floats
   static constexpr int kScan = (kThreads / 32) * (1 + NS) * kSlab * 4;
-  static constexpr int kStages = 2;                                        // chunk pipeline depth
-  static constexpr int kBytes = kStages * kData + kScan + 128;             // + alignment
+  static constexpr int kBytes = kData + kScan + 128;                       // + alignment
 };
 
-template <typename T, int NS>
+template <typename T, int NS, int R = kRows>
 __global__ void __launch_bounds__(kThreads, 2)
 scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x0,
             const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ Params<T, NS> p) {
-  using S = Shape<T>;
-  using SM = Smem<T, NS>;
-  constexpr int V = S::kVec, LANES = S::kLanes, L = S::kChunk;
+  using S = Shape<T, R>;
+  using SM = Smem<T, NS, R>;
+  constexpr int V = S::kVec, V2 = V / 2, LANES = S::kLanes, L = S::kChunk;
+  constexpr int NW = kThreads / 32;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
-  constexpr int NW = kThreads / 32;
-  constexpr int NSTG = SM::kStages;
-  float* s_w = reinterpret_cast<float*>(smem + NSTG * SM::kData);    // [NW][1 + NS][64]
-  __shared__ __align__(8) uint64_t s_bar[NSTG];
-  __shared__ unsigned int s_ticket[NSTG];
+  const T* s_g = reinterpret_cast<const T*>(smem);
+  float* s_w = reinterpret_cast<float*>(smem + SM::kData);            // [NW][1 + NS][64]
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ unsigned int s_ticket;
   __shared__ float s_tot_a[kSlab];
   __shared__ float s_tot_b[NS][kSlab];
   __shared__ float s_carry[NS][kSlab];
   static_assert(32 % LANES == 0, "row groups of a warp must share channels");
 
   const int tid = threadIdx.x;
-  const unsigned int n_total = (unsigned int)p.n_chains * (unsigned int)p.n_chunks_t;
-  // TMA loads of chunk `tk` (gate tile first) into pipeline stage `stg`;
-  // rows past T read as zero
-  auto fetch = [&](unsigned int tk, int stg) {
-    const int ck = tk / p.n_chains, chn = tk % p.n_chains;
-    const uint32_t bb = sm100::smem_u32(&s_bar[stg]);
-    sm100::mbar_arrive_expect_tx(bb, SM::kData);
-    const uint32_t dst = sm100::smem_u32(smem + stg * SM::kData);
-    const int x = (chn % p.slabs) * kSlab, y = ck * L, z = chn / p.slabs;
-    sm100::tma_load_3d(dst, &tm_g, bb, x, y, z);
-    sm100::tma_load_3d(dst + SM::kTile, &tm_x0, bb, x, y, z);
-    if (NS == 2) sm100::tma_load_3d(dst + 2 * SM::kTile, &tm_x1, bb, x, y, z);
-  };
   auto aborted = [&]() -> bool {
     unsigned int v;
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.ws.abort) : "memory");
     return v != 0u;
   };
+  const uint32_t bar = sm100::smem_u32(&s_bar);
   if (tid == 0) {
-    for (int i = 0; i < NSTG; ++i) sm100::mbar_init(sm100::smem_u32(&s_bar[i]), 1);
+    s_ticket = atomicAdd(p.ws.counter, 1u);
+    sm100::mbar_init(bar, 1);
     sm100::fence_barrier_init();
-    const unsigned int tk = atomicAdd(p.ws.counter, 1u);
-    s_ticket[0] = tk;
-    if (tk < n_total) fetch(tk, 0);
   }
   __syncthreads();
-
-  // Persistent loop: chunk tickets come in launch order; while this CTA scans
-  // one chunk, the next ticket's tiles are already being loaded.
-  for (int it = 0;; ++it) {
-  const int stage = it & 1;
-  const unsigned int ticket = s_ticket[stage];
-  if (ticket >= n_total) break;
-  if (tid == 0) {
-    const unsigned int nx = atomicAdd(p.ws.counter, 1u);
-    s_ticket[stage ^ 1] = nx;
-    if (nx < n_total) fetch(nx, stage ^ 1);
-  }
-  const T* s_g = reinterpret_cast<const T*>(smem + stage * SM::kData);
-  const int chunk = ticket / p.n_chains;     // chunk-major: predecessors were ticketed earlier
+  const unsigned int ticket = s_ticket;
+  const int chunk = ticket / p.n_chains;     // chunk-major: predecessors started earlier
   const int chain = ticket % p.n_chains;
   const int b = chain / p.slabs;
   const int slab = chain % p.slabs;
   const long long desc = (long long)chain * p.n_chunks_t + chunk;   // descriptor index
 
+  // ---- TMA: gate and input tiles of this chunk (rows past T read as zero) ----
+  if (tid == 0) {
+    sm100::mbar_arrive_expect_tx(bar, SM::kData);
+    const uint32_t dst = sm100::smem_u32(smem);
+    sm100::tma_load_3d(dst, &tm_g, bar, slab * kSlab, chunk * L, b);
+    sm100::tma_load_3d(dst + SM::kTile, &tm_x0, bar, slab * kSlab, chunk * L, b);
+    if (NS == 2) sm100::tma_load_3d(dst + 2 * SM::kTile, &tm_x1, bar, slab * kSlab, chunk * L, b);
+  }
+
   const int lane_c = tid % LANES;            // 16-byte column within the slab
   const int grp = tid / LANES;               // row group
-  const int t0 = chunk * L + grp * kRows;    // first token of this thread
-  const int nrows = max(0, min(kRows, p.Tn - t0));   // valid tokens of this thread
+  const int t0 = chunk * L + grp * R;        // first token of this thread
+  const int nrows = max(0, min(R, p.Tn - t0));   // valid tokens of this thread
   const long long row_stride = p.C;
   const long long base = ((long long)b * p.Tn) * row_stride + (long long)slab * kSlab + lane_c * V;
-  const int soff = grp * kRows * kSlab + lane_c * V;   // element offset of row 0 in a tile
+  const int soff = grp * R * kSlab + lane_c * V;   // element offset of row 0 in a tile
 
   {
     // one thread waits for the tiles (bounded; the clock and the abort word
     // are read every 64 polls), the others sleep in the barrier
     bool ok = true;
     if (tid == 0) {
-      const uint32_t bb = sm100::smem_u32(&s_bar[stage]);
       unsigned long long tw = 0;
       unsigned int n = 0;
-      while (!sm100::mbar_try_wait(bb, (it >> 1) & 1)) {
+      while (!sm100::mbar_try_wait(bar, 0)) {
         if ((++n & 63u) == 0u) {
           const unsigned long long now = global_ns();
           if (tw == 0) tw = now;
@@ -220,8 +203,8 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
       }
     }
     if (!__syncthreads_and(ok)) {
-      // give up: publish a zero state for this chunk, make every other CTA
-      // stop waiting, and leave
+      // give up: publish a zero state for this chunk and make every other
+      // CTA stop waiting
       if (tid < 32) {
 #pragma unroll
         for (int w = 0; w < 2 * NS; ++w)
@@ -229,55 +212,49 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
         if (tid == 0) {
           raise_error(RATP_ERR_TIMEOUT);
           atomicExch(p.ws.abort, 1u);
-          // let the prefetch into the other stage land before the CTA exits
-          if (s_ticket[stage ^ 1] < n_total) {
-            const uint32_t bo = sm100::smem_u32(&s_bar[stage ^ 1]);
-            const unsigned long long t1 = global_ns();
-            while (!sm100::mbar_try_wait(bo, ((it + 1) >> 1) & 1) && global_ns() - t1 < spin_timeout()) {
-            }
-          }
         }
       }
-      break;
+      return;
     }
   }
 
-  // ---- thread-local aggregate of its tokens ----
-  float la[V], lb[NS][V];
+  // ---- thread-local aggregate of its tokens (channel pairs) ----
+  float2 la[V2], lb[NS][V2];
 #pragma unroll
-  for (int i = 0; i < V; ++i) la[i] = 1.f;
+  for (int i = 0; i < V2; ++i) {
+    la[i] = make_float2(1.f, 1.f);
 #pragma unroll
-  for (int s = 0; s < NS; ++s)
+    for (int s = 0; s < NS; ++s) lb[s][i] = make_float2(0.f, 0.f);
+  }
 #pragma unroll
-    for (int i = 0; i < V; ++i) lb[s][i] = 0.f;
-#pragma unroll
-  for (int r = 0; r < kRows; ++r) {
+  for (int r = 0; r < R; ++r) {
     if (r < nrows) {
-      float gf[V];
-      Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_g + soff + r * kSlab), gf);
+      float2 gf[V2];
+      Elem<T>::unpack2(*reinterpret_cast<const uint4*>(s_g + soff + r * kSlab), gf);
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        float xf[V];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_g + (1 + s) * L * kSlab + soff + r * kSlab), xf);
+        float2 xf[V2];
+        Elem<T>::unpack2(*reinterpret_cast<const uint4*>(s_g + (1 + s) * L * kSlab + soff + r * kSlab), xf);
 #pragma unroll
-        for (int i = 0; i < V; ++i) lb[s][i] = fmaf(gf[i], lb[s][i] - xf[i], xf[i]);
+        for (int i = 0; i < V2; ++i) lb[s][i] = fma2(gf[i], sub2(lb[s][i], xf[i]), xf[i]);
       }
 #pragma unroll
-      for (int i = 0; i < V; ++i) la[i] *= gf[i];
+      for (int i = 0; i < V2; ++i) la[i] = mul2(la[i], gf[i]);
     }
   }
+
   // ---- intra-chunk scan over row groups, hierarchical ----
   // (1) the row groups of one warp hold the same channels in lanes
   //     lane_c, lane_c + LANES, ...: a shuffle scan over them (stride LANES)
   //     gives each thread the map of the warp's rows up to and including its
   //     own; (2) lane group GW-1 publishes the warp total, warp 0 scans the NW
-  //     totals per channel; (3) each thread composes the exclusive prefix.
+  //     totals per channel; (3) each thread composes its exclusive prefix.
   constexpr int GW = 32 / LANES;             // row groups per warp
   const int lane = tid & 31, wid = tid >> 5;
   const int gw = lane / LANES;               // row group within the warp
-  float ia[V], ib[NS][V];                    // inclusive map within the warp
+  float2 ia[V2], ib[NS][V2];                 // inclusive map within the warp
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
+  for (int i = 0; i < V2; ++i) {
     ia[i] = la[i];
 #pragma unroll
     for (int s = 0; s < NS; ++s) ib[s][i] = lb[s][i];
@@ -285,77 +262,86 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
 #pragma unroll
   for (int d = 1; d < GW; d <<= 1) {
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-      const float ua = __shfl_up_sync(0xffffffffu, ia[i], d * LANES);
-      float ub[NS];
+    for (int i = 0; i < V2; ++i) {
+      float2 ua, ub[NS];
+      ua.x = __shfl_up_sync(0xffffffffu, ia[i].x, d * LANES);
+      ua.y = __shfl_up_sync(0xffffffffu, ia[i].y, d * LANES);
 #pragma unroll
-      for (int s = 0; s < NS; ++s) ub[s] = __shfl_up_sync(0xffffffffu, ib[s][i], d * LANES);
+      for (int s = 0; s < NS; ++s) {
+        ub[s].x = __shfl_up_sync(0xffffffffu, ib[s][i].x, d * LANES);
+        ub[s].y = __shfl_up_sync(0xffffffffu, ib[s][i].y, d * LANES);
+      }
       if (gw >= d) {
 #pragma unroll
-        for (int s = 0; s < NS; ++s) ib[s][i] = fmaf(ia[i], ub[s], ib[s][i]);   // self o up
-        ia[i] *= ua;
+        for (int s = 0; s < NS; ++s) ib[s][i] = fma2(ia[i], ub[s], ib[s][i]);   // self o up
+        ia[i] = mul2(ia[i], ua);
       }
     }
   }
   if (gw == GW - 1) {                        // warp total
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-      s_w[(wid * (1 + NS)) * kSlab + lane_c * V + i] = ia[i];
+    for (int i = 0; i < V2; ++i) {
+      const int c = lane_c * V + 2 * i;
+      *reinterpret_cast<float2*>(s_w + (wid * (1 + NS)) * kSlab + c) = ia[i];
 #pragma unroll
-      for (int s = 0; s < NS; ++s) s_w[(wid * (1 + NS) + 1 + s) * kSlab + lane_c * V + i] = ib[s][i];
+      for (int s = 0; s < NS; ++s) *reinterpret_cast<float2*>(s_w + (wid * (1 + NS) + 1 + s) * kSlab + c) = ib[s][i];
     }
   }
   __syncthreads();
   if (tid < 32) {
     // exclusive prefix over warps (in place) and the chunk total, 2 channels per lane
+    const int c = 2 * tid;
+    float2 pa = make_float2(1.f, 1.f), pb[NS];
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-      const int c = 2 * tid + cc;
-      float pa = 1.f, pb[NS];
+    for (int s = 0; s < NS; ++s) pb[s] = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int s = 0; s < NS; ++s) pb[s] = 0.f;
+    for (int w = 0; w < NW; ++w) {
+      float2* wa = reinterpret_cast<float2*>(s_w + (w * (1 + NS)) * kSlab + c);
+      const float2 va = *wa;
+      *wa = pa;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        const float wa = s_w[(w * (1 + NS)) * kSlab + c];
-        float wb[NS];
-#pragma unroll
-        for (int s = 0; s < NS; ++s) wb[s] = s_w[(w * (1 + NS) + 1 + s) * kSlab + c];
-        s_w[(w * (1 + NS)) * kSlab + c] = pa;
-#pragma unroll
-        for (int s = 0; s < NS; ++s) {
-          s_w[(w * (1 + NS) + 1 + s) * kSlab + c] = pb[s];
-          pb[s] = fmaf(wa, pb[s], wb[s]);    // warp w applied after the prefix
-        }
-        pa *= wa;
+      for (int s = 0; s < NS; ++s) {
+        float2* wb = reinterpret_cast<float2*>(s_w + (w * (1 + NS) + 1 + s) * kSlab + c);
+        const float2 vb = *wb;
+        *wb = pb[s];
+        pb[s] = fma2(va, pb[s], vb);         // warp w applied after the prefix
       }
-      s_tot_a[c] = pa;
+      pa = mul2(pa, va);
+    }
+    s_tot_a[c] = pa.x;
+    s_tot_a[c + 1] = pa.y;
 #pragma unroll
-      for (int s = 0; s < NS; ++s) s_tot_b[s][c] = pb[s];
+    for (int s = 0; s < NS; ++s) {
+      s_tot_b[s][c] = pb[s].x;
+      s_tot_b[s][c + 1] = pb[s].y;
     }
   }
   __syncthreads();
-  // exclusive map of this thread's row group: (inclusive within warp minus
-  // own group) composed after the warp prefix
-  float ea[V], eb[NS][V];
+  // exclusive map of this thread's row group: (within-warp exclusive) o (warp prefix)
+  float2 ea[V2], eb[NS][V2];
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    // within-warp exclusive = the inclusive map of the row group above (gw - 1)
-    float xa = __shfl_up_sync(0xffffffffu, ia[i], LANES);
-    float xb[NS];
-#pragma unroll
-    for (int s = 0; s < NS; ++s) xb[s] = __shfl_up_sync(0xffffffffu, ib[s][i], LANES);
-    if (gw == 0) {
-      xa = 1.f;
-#pragma unroll
-      for (int s = 0; s < NS; ++s) xb[s] = 0.f;
-    }
-    const float wa = s_w[(wid * (1 + NS)) * kSlab + lane_c * V + i];
+  for (int i = 0; i < V2; ++i) {
+    float2 xa, xb[NS];
+    xa.x = __shfl_up_sync(0xffffffffu, ia[i].x, LANES);
+    xa.y = __shfl_up_sync(0xffffffffu, ia[i].y, LANES);
 #pragma unroll
     for (int s = 0; s < NS; ++s) {
-      const float wb = s_w[(wid * (1 + NS) + 1 + s) * kSlab + lane_c * V + i];
-      eb[s][i] = fmaf(xa, wb, xb[s]);        // (within-warp exclusive) o (warp prefix)
+      xb[s].x = __shfl_up_sync(0xffffffffu, ib[s][i].x, LANES);
+      xb[s].y = __shfl_up_sync(0xffffffffu, ib[s][i].y, LANES);
     }
-    ea[i] = xa * wa;
+    if (gw == 0) {
+      xa = make_float2(1.f, 1.f);
+#pragma unroll
+      for (int s = 0; s < NS; ++s) xb[s] = make_float2(0.f, 0.f);
+    }
+    const int c = lane_c * V + 2 * i;
+    const float2 wa = *reinterpret_cast<const float2*>(s_w + (wid * (1 + NS)) * kSlab + c);
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const float2 wb = *reinterpret_cast<const float2*>(s_w + (wid * (1 + NS) + 1 + s) * kSlab + c);
+      eb[s][i] = fma2(xa, wb, xb[s]);
+    }
+    ea[i] = mul2(xa, wa);
   }
 
   // ---- publish, look back, publish inclusive (warp 0) ----
@@ -475,36 +461,34 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   __syncthreads();
 
   // ---- recompute the tokens from the carry and store ----
-  float hs[NS][V];
+  float2 hs[NS][V2];
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const int c = lane_c * V + i;
+  for (int i = 0; i < V2; ++i) {
+    const int c = lane_c * V + 2 * i;
 #pragma unroll
-    for (int s = 0; s < NS; ++s) hs[s][i] = fmaf(ea[i], s_carry[s][c], eb[s][i]);
+    for (int s = 0; s < NS; ++s) hs[s][i] = fma2(ea[i], make_float2(s_carry[s][c], s_carry[s][c + 1]), eb[s][i]);
   }
 #pragma unroll
-  for (int r = 0; r < kRows; ++r) {
+  for (int r = 0; r < R; ++r) {
     if (r < nrows) {
       const int t = t0 + r;
-      float gf[V];
-      Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_g + soff + r * kSlab), gf);
+      float2 gf[V2];
+      Elem<T>::unpack2(*reinterpret_cast<const uint4*>(s_g + soff + r * kSlab), gf);
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        float xf[V];
-        Elem<T>::unpack(*reinterpret_cast<const uint4*>(s_g + (1 + s) * L * kSlab + soff + r * kSlab), xf);
+        float2 xf[V2];
+        Elem<T>::unpack2(*reinterpret_cast<const uint4*>(s_g + (1 + s) * L * kSlab + soff + r * kSlab), xf);
 #pragma unroll
-        for (int i = 0; i < V; ++i) hs[s][i] = fmaf(gf[i], hs[s][i] - xf[i], xf[i]);
+        for (int i = 0; i < V2; ++i) hs[s][i] = fma2(gf[i], sub2(hs[s][i], xf[i]), xf[i]);
         const long long off = base + (long long)t * row_stride;
-        __stcs(reinterpret_cast<uint4*>(p.h[s] + off), Elem<T>::pack(hs[s]));
+        __stcs(reinterpret_cast<uint4*>(p.h[s] + off), Elem<T>::pack2(hs[s]));
         if (t == p.Tn - 1 && p.final_state != nullptr) {
           float* fs = p.final_state + ((long long)s * p.B + b) * p.C + slab * kSlab + lane_c * V;
 #pragma unroll
-          for (int i = 0; i < V; ++i) fs[i] = hs[s][i];
+          for (int i = 0; i < V2; ++i) { fs[2 * i] = hs[s][i].x; fs[2 * i + 1] = hs[s][i].y; }
         }
       }
     }
-  }
-  __syncthreads();   // stage and ticket slot may be refilled from here on
   }
 }
 

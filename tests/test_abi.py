@@ -65,8 +65,10 @@ def test_status_strings(lib):
 def test_scan_workspace_query(lib):
     n = ctypes.c_size_t()
     assert lib.ratp_scan_workspace_bytes(8, 4096, 16, 128, 1, ctypes.byref(n)) == 0
-    chunks = 8 * (2048 // 64) * (4096 // 128)
-    assert n.value >= chunks * (4 + 4 * 64 * 5)
+    # bf16 chunks of 256 tokens x 64 channels; per chunk 32 lanes x 64-bit
+    # words: 2 x (1 + 2) aggregate words and 2 x 2 inclusive words
+    chunks = 8 * (2048 // 64) * (4096 // 256)
+    assert n.value >= chunks * 32 * 8 * (2 * 3 + 2 * 2)
     assert lib.ratp_scan_workspace_bytes(1, 10, 1, 32, 1, ctypes.byref(n)) == 2   # H*Dh % 64
     assert lib.ratp_scan_workspace_bytes(-1, 10, 1, 64, 1, ctypes.byref(n)) == 1
     assert lib.ratp_scan_workspace_bytes(1, 10, 1, 64, 7, ctypes.byref(n)) == 1
