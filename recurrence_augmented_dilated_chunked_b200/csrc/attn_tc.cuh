@@ -1,5 +1,5 @@
 // attn_tc.cuh -- dilated (+ windowed) prefill attention on the 5th-generation
-// tensor cores (TMA + tcgen05.mma, accumulators in tensor memory).
+// tensor cores (TMA + tcgen05.mma, accumulators and P in tensor memory).
 //
 // Computes, for every (b, h, t), softmax attention of q[b,t,h] over the
 // recurrent keys/values at K_h(t) = {j < t : j mod D_h = D_h-1} U {t}
@@ -18,31 +18,36 @@
 // Each key is counted once by splitting the set at the window: row t takes
 // every window position t-W'+1..t and only the dilated slots whose position
 // lies before the window, s < floor((t - W' + 1) / D).  So per-row validity is
-// a prefix (dilated; dense: s <= t) or a contiguous range (window), evaluated
-// as bit masks per 32-column chunk.
+// a prefix (dilated; dense: s <= t) or a contiguous range (window), applied as
+// bit masks per 32-column chunk.
 //
-// Roles (352 threads, one CTA per SM, persistent over items in heavy-first
-// order -- dense heads and late query tiles first, round-robin over CTAs):
-//   warps 0-7  softmax: warps w and w+4 share query rows 32(w%4)..+31 (TMEM
-//              lanes) and split the 128 key columns in halves.  Each reads its
-//              half of S from TMEM, masks it per 32-column chunk with a bit
-//              mask (all-valid and all-masked chunks take fast paths), the
-//              pair exchanges the row max through shared memory, the running
-//              max is kept with O rescaled in TMEM only when it grows by more
-//              than 2^8, and P (bf16) is written into one of two 128B-swizzled
-//              K-major smem tiles.  An item's epilogue (normalise half an O
-//              row, store) runs after the softmax of the next item's first
-//              tile, so waiting for its last P V overlaps useful work.
-//   warp 8     TMA producer of Q and of a 2-stage K ring (a K stage is freed
-//              as soon as its S = Q K^T completes);
-//   warp 10    TMA producer of a 2-stage V ring (freed when P V completes);
-//   warp 9     allocates TMEM (512 columns: S ping-pong 2x128, O ping-pong
-//              2x128, one O per work item in flight) and one
-//              lane issues S = Q K^T (SS, K-major) and O += P V (P K-major,
-//              V MN-major) as 128x128x16 tcgen05.mma; completions signal
-//              mbarriers via tcgen05.commit.
+// Two CTAs per SM, persistent over items blockIdx.x, +G, +2G, ... (G = grid
+// size = 2 x SMs; items in heavy-first order: dense heads and late query tiles
+// first).  A CTA runs one item at a time as a chain per key tile:
+// S = Q K^T -> softmax -> O += P V; the other CTA on the SM fills the tensor
+// core while this one is in its softmax.  Because each CTA's chain is
+// serial, one buffer each of Q, K and V (96 KB) hides the loads: K of tile
+// n+1 is fetched while tile n is in softmax and P V, V of tile n+1 while
+// tile n+1 is in S = Q K^T and softmax, and the next item's Q while the last
+// tile finishes.  A tcgen05.mma of M=128 with N >= 128 runs at the tensor
+// core's full rate; the issuing thread keeps its instruction stream between
+// MMAs to precomputed descriptor additions.
+//
+// Roles (192 threads per CTA):
+//   warps 0-3  softmax: one thread per query row (warp w reads TMEM lanes
+//              32w..32w+31), all 128 key columns of the row.  Reads S from
+//              TMEM, masks, takes the row max, writes P = 2^(s - m) as bf16
+//              pairs over the first 64 columns of S, rescales O in TMEM only
+//              when the running max grew by more than 2^8, and after the
+//              item's last tile normalises O and stores the output rows.
+//   warp 4     one lane: TMA producer of Q, K and V;
+//   warp 5     allocates TMEM (256 columns: S/P at 0, O at 128) and one lane
+//              issues S = Q K^T (M=128, N=128, K=128; Q and K K-major in
+//              smem) and O += P V (M=128, N=128, K=128; P K-major in TMEM, V
+//              MN-major in smem) as tcgen05.mma with K=16 steps.
 // Every mbarrier wait is bounded; on expiry the CTA records RATP_ERR_TIMEOUT,
-// all roles drain out, and TMEM is released.
+// all roles drain out (copies and MMAs in flight are waited for), and TMEM
+// is released.
 #pragma once
 #include "sm100.cuh"
 
@@ -52,27 +57,25 @@ namespace attn_tc {
 constexpr int BM = 128;          // queries per tile
 constexpr int BN = 128;          // keys per tile
 constexpr int DH = 128;          // head dim
-constexpr int NST = 2;           // K/V pipeline stages
-constexpr int kSoftmaxWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kVProducerWarp = 10;
-constexpr int kThreads = 352;
-constexpr uint32_t kHalf = BN * 64 * 2;        // one 64-column half tile: 16 KB
+constexpr int kCtasPerSm = 2;
+constexpr int kSoftmaxWarps = 4;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kThreads = 192;
+constexpr uint32_t kHalf = 128 * 64 * 2;       // 128 rows x 64 columns: 16 KB
 constexpr uint32_t kTile = 2 * kHalf;          // 128 x 128 bf16: 32 KB
-constexpr uint32_t kOffQ = 0;                  // Q
+constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kTile;
-constexpr uint32_t kOffV = kOffK + NST * kTile;
-constexpr uint32_t kOffP = kOffV + NST * kTile;  // 2 P buffers
-constexpr uint32_t kOffBar = kOffP + 2 * kTile;
-constexpr uint32_t kNumBars = 18;
-constexpr uint32_t kOffXchg = kOffBar + kNumBars * 8 + 16;     // row-max / row-sum exchange
-constexpr uint32_t kXchgBytes = 2 * BM * 4;                    // [2 halves][128] f32
-constexpr uint32_t kSmemBytes = kOffXchg + kXchgBytes + 1024;  // + alignment slack
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;      // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 256;    // O double buffer at columns 256..383 and 384..511
+constexpr uint32_t kOffV = kOffK + kTile;
+constexpr uint32_t kOffBar = kOffV + kTile;
+// barriers: qfull kfull vfull sfull pfull pvdone final
+constexpr uint32_t kNumBars = 7;
+constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + TMEM slot, abort, alignment
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0;      // S, then P over its first 64 columns
+constexpr uint32_t kColO = 128;    // O
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
 struct Params {
   __nv_bfloat16* o;
@@ -125,7 +128,8 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
   return it;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             const __grid_constant__ CUtensorMap tm_kpos,
             const __grid_constant__ CUtensorMap tm_vpos,
@@ -137,41 +141,29 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
-  const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV, sP = sb + kOffP;
+  const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV;
   const uint32_t bar0 = sb + kOffBar;
-  // barrier map
-  const uint32_t b_qfull = bar0 + 0 * 8;
-  const uint32_t b_qempty = bar0 + 1 * 8;
-  const uint32_t b_kfull = bar0 + 2 * 8;    // [NST]
-  const uint32_t b_kempty = bar0 + 4 * 8;   // [NST]
-  const uint32_t b_sfull = bar0 + 6 * 8;    // [2]
-  const uint32_t b_sfree = bar0 + 8 * 8;    // [2]
-  const uint32_t b_pfull = bar0 + 10 * 8;   // [2]
-  const uint32_t b_pvdone = bar0 + 12 * 8;  // [2]
-  const uint32_t b_vfull = bar0 + 14 * 8;   // [NST]
-  const uint32_t b_vempty = bar0 + 16 * 8;  // [NST]
+  const uint32_t b_qfull = bar0 + 0 * 8;    // Q landed
+  const uint32_t b_kfull = bar0 + 1 * 8;    // K landed
+  const uint32_t b_vfull = bar0 + 2 * 8;    // V landed
+  const uint32_t b_sfull = bar0 + 3 * 8;    // S = Q K^T done (K and, at an item's end, Q free)
+  const uint32_t b_pfull = bar0 + 4 * 8;    // P written (128 softmax threads)
+  const uint32_t b_pvdone = bar0 + 5 * 8;   // O += P V done (V, S/P free; O current)
+  const uint32_t b_final = bar0 + 6 * 8;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 4);
-  float* s_xchg = reinterpret_cast<float*>(smem + kOffXchg);     // [2 halves][128 rows]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
-    mbar_init(b_qempty, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(b_sfull + 8 * i, 1);
-      mbar_init(b_sfree + 8 * i, kSoftmaxWarps * 32);
-      mbar_init(b_pfull + 8 * i, kSoftmaxWarps * 32);
-      mbar_init(b_pvdone + 8 * i, 1);
-    }
-    for (int i = 0; i < NST; ++i) {
-      mbar_init(b_kfull + 8 * i, 1);
-      mbar_init(b_kempty + 8 * i, 1);
-      mbar_init(b_vfull + 8 * i, 1);
-      mbar_init(b_vempty + 8 * i, 1);
-    }
+    mbar_init(b_kfull, 1);
+    mbar_init(b_vfull, 1);
+    mbar_init(b_sfull, 1);
+    mbar_init(b_pfull, kSoftmaxWarps * 32);
+    mbar_init(b_pvdone, 1);
+    mbar_init(b_final, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -191,137 +183,217 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  if (warp == kProducerWarp || warp == kVProducerWarp) {
-    // ------------------------------------------------------------ producers
-    // warp kProducerWarp: Q and K tiles; warp kVProducerWarp: V tiles.  Both
-    // walk the same item/tile sequence.
-    const bool is_k = (warp == kProducerWarp);
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------ producer
+    // Tile n: Q (at an item's first tile) and K once S = Q K^T of tile n-1
+    // is done, V once O += P V of tile n-1 is done.
     if (lane == 0) {
-      const uint32_t ring = is_k ? sK : sV;
-      const uint32_t b_full = is_k ? b_kfull : b_vfull;
-      const uint32_t b_empty = is_k ? b_kempty : b_vempty;
-      int g = 0, li = 0;
+      int n = 0, nq = 0;                // tiles and Q loads issued
+      int last_k = -1, last_v = -1;     // tile of the last K / V load issued
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
+      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
         const Item it = make_item(p, idx);
-        if (is_k) {
-          if (li >= 1 && !mbar_wait(b_qempty, (li - 1) & 1, s_abort)) break;
-          mbar_arrive_expect_tx(b_qfull, kTile);
-          tma_load_4d(sQ, &tm_q, b_qfull, 0, it.h, it.t0, it.b);
-          tma_load_4d(sQ + kHalf, &tm_q, b_qfull, 64, it.h, it.t0, it.b);
-        }
-        for (int j = 0; j < it.n_tiles; ++j, ++g) {
-          const int st = g % NST;
-          if (g >= NST && !mbar_wait(b_empty + 8 * st, ((g / NST) - 1) & 1, s_abort)) {
-            ok = false;
-            break;
+        for (int j = 0; j < it.n_tiles; ++j, ++n) {
+          if (n > 0 && !mbar_wait(b_sfull, (n - 1) & 1, s_abort)) { ok = false; break; }
+          if (j == 0) {
+            mbar_arrive_expect_tx(b_qfull, kTile);
+            tma_load_4d(sQ, &tm_q, b_qfull, 0, it.h, it.t0, it.b);
+            tma_load_4d(sQ + kHalf, &tm_q, b_qfull, 64, it.h, it.t0, it.b);
+            ++nq;
           }
-          const CUtensorMap* m;
-          int row;
-          if (j < it.n_win) {
-            m = is_k ? &tm_kpos : &tm_vpos;
-            row = it.p_start + j * BN;
-          } else {
-            row = (j - it.n_win) * BN;
-            if (it.dense) m = is_k ? &tm_kpos : &tm_vpos;
-            else m = is_k ? &tm_kdil : &tm_vdil;
+          const bool pos = (j < it.n_win) || it.dense;
+          const int row = (j < it.n_win) ? it.p_start + j * BN : (j - it.n_win) * BN;
+          if (!(blockIdx.x == 0 && (long long)n == g_fault_attn_ktile)) {   // else: planted failure
+            const CUtensorMap* m = pos ? &tm_kpos : &tm_kdil;
+            mbar_arrive_expect_tx(b_kfull, kTile);
+            tma_load_4d(sK, m, b_kfull, 0, it.h, row, it.b);
+            tma_load_4d(sK + kHalf, m, b_kfull, 64, it.h, row, it.b);
+            last_k = n;
           }
-          if (is_k && blockIdx.x == 0 && (long long)g == g_fault_attn_ktile) continue;   // planted failure
-          const uint32_t fb = b_full + 8 * st;
-          mbar_arrive_expect_tx(fb, kTile);
-          tma_load_4d(ring + st * kTile, m, fb, 0, it.h, row, it.b);
-          tma_load_4d(ring + st * kTile + kHalf, m, fb, 64, it.h, row, it.b);
+          if (n > 0 && !mbar_wait(b_pvdone, (n - 1) & 1, s_abort)) { ok = false; break; }
+          const CUtensorMap* m = pos ? &tm_vpos : &tm_vdil;
+          mbar_arrive_expect_tx(b_vfull, kTile);
+          tma_load_4d(sV, m, b_vfull, 0, it.h, row, it.b);
+          tma_load_4d(sV + kHalf, m, b_vfull, 64, it.h, row, it.b);
+          last_v = n;
         }
       }
+      // let the copies in flight land before the CTA ends (after an abort
+      // they may never have been consumed): the last Q, K and V load
+      if (nq > 0) mbar_drain(b_qfull, (nq - 1) & 1);
+      if (last_k >= 0) mbar_drain(b_kfull, last_k & 1);
+      if (last_v >= 0) mbar_drain(b_vfull, last_v & 1);
     }
+    __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);    // Q K^T: both K-major
-      constexpr uint32_t idPV = idesc_bf16_f32(BM, DH, 0, 1);   // P V: V is MN-major
-      int g = 0, li = 0;
-      bool pend = false;
-      int pg = 0, pst = 0, pacc = 0, pob = 0;
+      constexpr uint32_t idPV = idesc_bf16_f32(BM, DH, 0, 1);   // P V: P K-major (TMEM), V MN-major
+      const uint64_t dq = sw128_desc(sQ, 16, 1024);
+      const uint64_t dk = sw128_desc(sK, 16, 1024);
+      const uint64_t dv = sw128_desc(sV, kHalf, 1024);
+      const uint32_t tS = tmem + kColS, tO = tmem + kColO;
+      int n = 0, li = 0;
       bool ok = true;
-      auto issue_pv = [&](int gg, int stg, int acc, int ob) -> bool {
-        const int pb = gg & 1;
-        if (!mbar_wait(b_pfull + 8 * pb, (gg >> 1) & 1, s_abort)) return false;
-        if (!mbar_wait(b_vfull + 8 * stg, (gg / NST) & 1, s_abort)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int k = 0; k < BN / 16; ++k) {
-          const uint64_t a = sw128_desc(sP + pb * kTile + (k >> 2) * kHalf + (k & 3) * 32, 16, 1024);
-          const uint64_t bdesc = sw128_desc(sV + stg * kTile + k * 16 * 128, kHalf, 1024);
-          umma_f16(tmem + kColO + ob * DH, a, bdesc, idPV, (acc || k > 0) ? 1u : 0u);
-        }
-        umma_commit(b_vempty + 8 * stg);
-        umma_commit(b_pvdone + 8 * pb);
-        return true;
-      };
       for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
-        const Item it = make_item(p, idx);
+        const int n_tiles = make_item(p, idx).n_tiles;
         if (!mbar_wait(b_qfull, li & 1, s_abort)) { ok = false; break; }
-        for (int j = 0; j < it.n_tiles; ++j, ++g) {
-          const int st = g % NST;
-          const int sbuf = g & 1;
-          if (!mbar_wait(b_kfull + 8 * st, (g / NST) & 1, s_abort)) { ok = false; break; }
-          if (g >= 2 && !mbar_wait(b_sfree + 8 * sbuf, ((g >> 1) - 1) & 1, s_abort)) { ok = false; break; }
+        for (int j = 0; j < n_tiles; ++j, ++n) {
+          // S/P columns are free once O += P V of tile n-1 is done
+          if (n > 0 && !mbar_wait(b_pvdone, (n - 1) & 1, s_abort)) { ok = false; break; }
+          if (!mbar_wait(b_kfull, n & 1, s_abort)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll
           for (int k = 0; k < DH / 16; ++k) {
-            const uint32_t koff = (k >> 2) * kHalf + (k & 3) * 32;
-            const uint64_t a = sw128_desc(sQ + koff, 16, 1024);
-            const uint64_t bdesc = sw128_desc(sK + st * kTile + koff, 16, 1024);
-            umma_f16(tmem + kColS + sbuf * BN, a, bdesc, idS, k > 0 ? 1u : 0u);
+            const uint64_t off = (uint64_t)(((k >> 2) * kHalf + (k & 3) * 32) >> 4);
+            umma_f16(tS, dq + off, dk + off, idS, k > 0 ? 1u : 0u);
           }
-          umma_commit(b_sfull + 8 * sbuf);
-          umma_commit(b_kempty + 8 * st);
-          if (j == it.n_tiles - 1) umma_commit(b_qempty);
-          if (pend && !issue_pv(pg, pst, pacc, pob)) { ok = false; break; }
-          pend = true;
-          pg = g; pst = st; pacc = (j > 0); pob = li & 1;
+          umma_commit(b_sfull);
+          if (!mbar_wait(b_pfull, n & 1, s_abort)) { ok = false; break; }
+          if (!mbar_wait(b_vfull, n & 1, s_abort)) { ok = false; break; }
+          tc_fence_after();
+          umma_f16_ts(tO, tS, dv, idPV, j > 0 ? 1u : 0u);
+#pragma unroll
+          for (int k = 1; k < BN / 16; ++k)
+            umma_f16_ts(tO, tS + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idPV, 1u);
+          umma_commit(b_pvdone);
         }
       }
-      if (ok && pend) issue_pv(pg, pst, pacc, pob);
+      // every MMA issued has completed before TMEM is released
+      umma_commit(b_final);
+      mbar_drain(b_final, 0);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    const int r = (warp & 3) * 32 + lane;            // query row within the tile (TMEM lane)
-    const int half = warp >> 2;                      // key/output column half
-    const int c_base = half * 64;
-    const uint32_t bar_id = 1 + (warp & 3);          // named barrier of the warp pair
-    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-    float* x_mine = s_xchg + half * BM + r;
-    const float* x_other = s_xchg + (1 - half) * BM + r;
-    auto pair_sync = [&]() {
-      asm volatile("bar.sync %0, %1;" :: "r"(bar_id), "r"(64) : "memory");
-    };
-    // The two warps of a pair meet at named barriers, so neither may leave the
-    // schedule early: after a failed (timed-out or aborted) wait the warps
-    // carry on with whatever tensor memory holds; every later wait fails fast
-    // and the error word already records the timeout.
-    // deferred epilogue of the previous item (-1: none): its item index, its
-    // O buffer, its last tile and this thread's partial row sum
-    int pend_idx = -1, pend_ob = 0, pend_gl = 0;
-    float pend_l = 0.f;
-    auto epilogue = [&](int e_idx, int e_ob, int e_gl, float e_l) {
-      const Item e = make_item(p, e_idx);
-      const int e_t = e.t0 + r;
-      warp_all(mbar_wait(b_pvdone + 8 * (e_gl & 1), (e_gl >> 1) & 1, s_abort));
-      tc_fence_after();
-      *x_mine = e_l;
-      pair_sync();
-      const float inv = 1.f / (e_l + *x_other);
-      pair_sync();
-      __nv_bfloat16* orow = p.o + (((size_t)e.b * p.T + e_t) * p.H + e.h) * DH + c_base;
-      const uint32_t ocol = kColO + e_ob * DH + c_base;
+    const int r = warp * 32 + lane;                  // query row within the tile (TMEM lane)
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t colS = tl + kColS, colO = tl + kColO;
+    const float sc = p.scale_log2;
+    // After a failed (timed-out or aborted) wait the warp leaves the loop;
+    // every wait is warp-uniform, so warp-collective tcgen05 instructions are
+    // always executed by the whole warp.
+    int n = 0;                                       // tiles so far
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+      const Item it = make_item(p, idx);
+      const int t = it.t0 + r;
+      const int lim_dil = it.dense ? (t + 1) : (max(0, t - p.W_eff + 1) / it.Dd);
+      const int w_lo = max(t - p.W_eff + 1, 0);
+      float m_used = -1e30f, l = 0.f;
+      for (int j = 0; j < it.n_tiles; ++j, ++n) {
+        // S of tile n; its completion also covers O += P V of tile n-1
+        if (!warp_all(mbar_wait(b_sfull, n & 1, s_abort))) { ok = false; break; }
+        tc_fence_after();
+        uint32_t sr[BN];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t o32[32];
-        tmem_ld32(tl + ocol + c * 32, o32);
+        for (int c = 0; c < 4; ++c) tmem_ld32(colS + 32 * c, sr + 32 * c);
         tmem_wait_ld();
-        if (e_t < p.T) {
+
+        // valid columns [lo, hi) of this row in this tile, as 32-bit chunk masks
+        int lo, hi;
+        if (j < it.n_win) {
+          const int base = it.p_start + j * BN;
+          lo = w_lo - base;
+          hi = t - base + 1;
+        } else {
+          lo = 0;
+          hi = lim_dil - (j - it.n_win) * BN;
+        }
+        uint32_t vm[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int clo = min(max(lo - 32 * c, 0), 32);
+          const int chi = min(max(hi - 32 * c, 0), 32);
+          vm[c] = (chi >= 32 ? 0xffffffffu : ((1u << chi) - 1u)) & ~(clo >= 32 ? 0xffffffffu : ((1u << clo) - 1u));
+        }
+        // mask in place (invalid -> -inf), then the row max of raw scores
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (!__all_sync(0xffffffffu, vm[c] == 0xffffffffu)) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              sr[32 * c + i] = ((vm[c] >> i) & 1u) ? sr[32 * c + i] : 0xff800000u;
+          }
+          float m3[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float a = __uint_as_float(sr[32 * c + i + 2 * u]);
+              const float b = __uint_as_float(sr[32 * c + i + 2 * u + 1]);
+              asm("max.f32 %0, %1, %2, %3;" : "=f"(m3[u]) : "f"(m3[u]), "f"(a), "f"(b));
+            }
+          }
+          float m01, m23;
+          asm("max.f32 %0, %1, %2, %3;" : "=f"(m01) : "f"(mx), "f"(m3[0]), "f"(m3[1]));
+          asm("max.f32 %0, %1, %2, %3;" : "=f"(m23) : "f"(m01), "f"(m3[2]), "f"(m3[3]));
+          mx = m23;
+        }
+        const float mxs = mx * sc;                   // -inf stays -inf
+        // O is rescaled only when some row's running max grew by more than
+        // 2^kRescaleThreshold; tcgen05.ld/st are warp-collective, so the
+        // decision is per warp and rows that do not need it scale by 1.
+        const bool need = (j > 0) && (mxs > m_used + kRescaleThreshold);
+        if (j == 0) m_used = fmaxf(mxs, -1e30f);
+        const bool rescale = __any_sync(0xffffffffu, need);
+        const float alpha = need ? exp2f(m_used - mxs) : 1.f;
+        if (need) {
+          l *= alpha;
+          m_used = mxs;
+        }
+        // p = 2^(s*scale - m) as bf16 pairs over S columns 16c..16c+15
+        const float2 sc2 = make_float2(sc, sc);
+        const float2 nm2 = make_float2(-m_used, -m_used);
+        float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t w[16];
+          if (__all_sync(0xffffffffu, vm[c] == 0u)) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = 0u;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 x = fma2(make_float2(__uint_as_float(sr[32 * c + 2 * i]),
+                                                __uint_as_float(sr[32 * c + 2 * i + 1])), sc2, nm2);
+              const float2 e = make_float2(exp2f(x.x), exp2f(x.y));
+              ls[i & 1] = add2(ls[i & 1], e);
+              w[i] = pack_bf16x2(e.x, e.y);
+            }
+          }
+          tmem_st16(colS + 16 * c, w);
+        }
+        l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+        if (rescale) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o32[32];
+            tmem_ld32(colO + 32 * c, o32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
+            tmem_st32(colO + 32 * c, o32);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(b_pfull);
+      }
+      if (!ok) break;
+      // epilogue: wait for the item's last P V, normalise, store
+      if (!warp_all(mbar_wait(b_pvdone, (n - 1) & 1, s_abort))) { ok = false; break; }
+      tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = p.o + (((size_t)it.b * p.T + t) * p.H + it.h) * DH;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o32[32];
+        tmem_ld32(colO + 32 * c, o32);
+        tmem_wait_ld();
+        if (t < p.T) {
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
             uint4 pk;
@@ -329,151 +401,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             pk.y = pack_bf16x2(__uint_as_float(o32[8 * v + 2]) * inv, __uint_as_float(o32[8 * v + 3]) * inv);
             pk.z = pack_bf16x2(__uint_as_float(o32[8 * v + 4]) * inv, __uint_as_float(o32[8 * v + 5]) * inv);
             pk.w = pack_bf16x2(__uint_as_float(o32[8 * v + 6]) * inv, __uint_as_float(o32[8 * v + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = pk;
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v) = pk;
           }
         }
       }
       tc_fence_before();
-    };
-    int g = 0, li = 0;
-    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x, ++li) {
-      const Item it = make_item(p, idx);
-      const int ob = li & 1;
-      const uint32_t ocol_item = kColO + ob * DH + c_base;
-      const int t = it.t0 + r;
-      const int lim_dil = it.dense ? (t + 1) : (max(0, t - p.W_eff + 1) / it.Dd);
-      const int w_lo = max(t - p.W_eff + 1, 0);
-      float m_used = -1e30f, l = 0.f;
-      for (int j = 0; j < it.n_tiles; ++j, ++g) {
-        const int sbuf = g & 1;
-        warp_all(mbar_wait(b_sfull + 8 * sbuf, (g >> 1) & 1, s_abort));
-        tc_fence_after();
-        uint32_t sr[64];
-        tmem_ld32(tl + kColS + sbuf * BN + c_base, sr);
-        tmem_ld32(tl + kColS + sbuf * BN + c_base + 32, sr + 32);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(b_sfree + 8 * sbuf);
-
-        // validity bit masks of the two 32-column chunks of this half
-        uint32_t vm[2];
-        {
-          const int lim_lo = (j < it.n_win) ? (w_lo - (it.p_start + j * BN) - c_base) : 0;
-          const int lim_hi = (j < it.n_win) ? (t - (it.p_start + j * BN) - c_base + 1)
-                                            : (lim_dil - (j - it.n_win) * BN - c_base);
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int lo = min(max(lim_lo - 32 * k, 0), 32);   // first valid column of the chunk
-            const int hi = min(max(lim_hi - 32 * k, 0), 32);   // one past the last valid column
-            vm[k] = (hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u)) & ~(lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u));
-          }
-        }
-        // masked row max of this half (raw scores)
-        // (four independent accumulators per chunk keep the chain short)
-        float mx = -INFINITY;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          if (vm[k] == 0xffffffffu) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) m4[i & 3] = fmaxf(m4[i & 3], __uint_as_float(sr[32 * k + i]));
-          } else if (vm[k] != 0u) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float v = __uint_as_float(sr[32 * k + i]);
-              m4[i & 3] = fmaxf(m4[i & 3], ((vm[k] >> i) & 1u) ? v : -INFINITY);
-            }
-          }
-          mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
-        }
-        // combine with the partner half of the row
-        *x_mine = mx;
-        pair_sync();
-        mx = fmaxf(mx, *x_other);
-        pair_sync();
-        const float mxs = mx * p.scale_log2;               // -inf stays -inf
-        // P buffer g&1 was last read by P.V of tile g-2
-        if (g >= 2) warp_all(mbar_wait(b_pvdone + 8 * sbuf, ((g >> 1) - 1) & 1, s_abort));
-        // O is rescaled only when some row's running max grew by more than
-        // 2^kRescaleThreshold; tcgen05.ld/st are warp-collective, so the
-        // decision is per warp (both warps of a pair decide alike) and rows
-        // that do not need it scale by 1.  P.V of tile g-1 must be complete.
-        const bool need = (j > 0) && (mxs > m_used + kRescaleThreshold);
-        if (j == 0) m_used = fmaxf(mxs, -1e30f);
-        if (__any_sync(0xffffffffu, need)) {
-          const int pb1 = (g - 1) & 1;
-          warp_all(mbar_wait(b_pvdone + 8 * pb1, ((g - 1) >> 1) & 1, s_abort));
-          tc_fence_after();
-          const float alpha = need ? exp2f(m_used - mxs) : 1.f;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t o32[32];
-            tmem_ld32(tl + ocol_item + c * 32, o32);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o32[i] = __float_as_uint(__uint_as_float(o32[i]) * alpha);
-            tmem_st32(tl + ocol_item + c * 32, o32);
-          }
-          tmem_wait_st();
-          if (need) {
-            l *= alpha;
-            m_used = mxs;
-          }
-        }
-        // p = 2^(s*scale - m), bf16 into the swizzled P tile (keys c_base..c_base+63)
-        const uint32_t prow = sP + sbuf * kTile + half * kHalf + r * 128;
-        const float neg_m = -m_used;
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          uint32_t w[16];
-          if (vm[k] == 0u) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = 0u;
-          } else if (vm[k] == 0xffffffffu) {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float e0 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i]), p.scale_log2, neg_m));
-              const float e1 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i + 1]), p.scale_log2, neg_m));
-              rs[i & 3] += e0 + e1;
-              w[i] = pack_bf16x2(e0, e1);
-            }
-          } else {
-            // exponentiate every column, then select: no per-element branches
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float e0 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i]), p.scale_log2, neg_m));
-              float e1 = exp2f(fmaf(__uint_as_float(sr[32 * k + 2 * i + 1]), p.scale_log2, neg_m));
-              e0 = ((vm[k] >> (2 * i)) & 1u) ? e0 : 0.f;
-              e1 = ((vm[k] >> (2 * i + 1)) & 1u) ? e1 : 0.f;
-              rs[i & 3] += e0 + e1;
-              w[i] = pack_bf16x2(e0, e1);
-            }
-          }
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint32_t chunk = (uint32_t)(4 * k + v);                 // 16-byte chunk in the half row
-            const uint32_t addr = prow + ((chunk ^ ((uint32_t)r & 7u)) << 4);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                         :: "r"(addr), "r"(w[4 * v]), "r"(w[4 * v + 1]), "r"(w[4 * v + 2]), "r"(w[4 * v + 3])
-                         : "memory");
-          }
-        }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(b_pfull + 8 * sbuf);
-        if (j == 0 && pend_idx >= 0) {
-          epilogue(pend_idx, pend_ob, pend_gl, pend_l);
-          pend_idx = -1;
-        }
-      }
-      pend_idx = idx;
-      pend_ob = ob;
-      pend_gl = g - 1;
-      pend_l = l;
     }
-    if (pend_idx >= 0) epilogue(pend_idx, pend_ob, pend_gl, pend_l);
   }
 
   tc_fence_before();

@@ -237,13 +237,13 @@ EncodeTiledFn encode_fn() {
 // [B][rows][H][128] bf16 view, rows of `row_stride_elems` elements apart,
 // starting `base_elems` elements into each batch item; box 64 x 1 x 128 x 1.
 bool make_map(CUtensorMap* m, const void* base, long long base_elems, int B, long long rows,
-              int H, long long row_stride_elems, long long batch_stride_elems) {
+              int H, long long row_stride_elems, long long batch_stride_elems, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[4] = {128, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
   const cuuint64_t strides[3] = {128 * 2, (cuuint64_t)row_stride_elems * 2,
                                  (cuuint64_t)batch_stride_elems * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   void* addr = const_cast<char*>(static_cast<const char*>(base)) + base_elems * 2;
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, addr, dims, strides, box, estr,
@@ -267,20 +267,22 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
   p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   const long long row = (long long)H * 128, bat = (long long)T * row;
   CUtensorMap tq, tkp, tvp, tkd, tvd;
-  if (!make_map(&tq, q, 0, B, T, H, row, bat) || !make_map(&tkp, hk, 0, B, T, H, row, bat) ||
-      !make_map(&tvp, hv, 0, B, T, H, row, bat))
+  constexpr int qr = attn_tc::BM, kr = attn_tc::BN;
+  if (!make_map(&tq, q, 0, B, T, H, row, bat, qr) || !make_map(&tkp, hk, 0, B, T, H, row, bat, kr) ||
+      !make_map(&tvp, hv, 0, B, T, H, row, bat, kr))
     return RATP_ERR_CUDA;
   const long long n_slots = T / D;
   if (n_slots >= 1) {
-    if (!make_map(&tkd, hk, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat) ||
-        !make_map(&tvd, hv, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat))
+    if (!make_map(&tkd, hk, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat, kr) ||
+        !make_map(&tvd, hv, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat, kr))
       return RATP_ERR_CUDA;
   } else {
     tkd = tkp;   // no dilated slot exists for any query: never read
     tvd = tvp;
   }
   if (!ensure_smem(attn_tc::attn_kernel, (int)attn_tc::kSmemBytes)) return RATP_ERR_CUDA;
-  const int grid = p.n_items < sm_count() ? p.n_items : sm_count();
+  const int slots = attn_tc::kCtasPerSm * sm_count();
+  const int grid = p.n_items < slots ? p.n_items : slots;
   attn_tc::attn_kernel<<<grid, attn_tc::kThreads, attn_tc::kSmemBytes, st>>>(tq, tkp, tvp, tkd, tvd, p);
   return launch_status();
 }
