@@ -7,9 +7,9 @@
 // windows; write-up section 6: dense heads D_h = 1).  bf16 in, fp32
 // accumulate, head dim 128.
 //
-// Work item = (b, h, 128-query tile).  Its keys come in 128-key tiles of two
+// Work item = (b, h, 128-query tile).  Its keys come in 64-key tiles of two
 // kinds, both fetched by plain tiled TMA boxes:
-//   * dilated tiles: slots s..s+127 of the strided view of hk/hv whose row s
+//   * dilated tiles: slots s..s+63 of the strided view of hk/hv whose row s
 //     is position s*D + D - 1 (base offset D-1 rows, row stride D rows), so the
 //     gather is an ordinary box of the strided tensor map; a dense head reads
 //     the positional view instead (slot = position);
@@ -23,28 +23,27 @@
 //
 // Two CTAs per SM, persistent over items blockIdx.x, +G, +2G, ... (G = grid
 // size = 2 x SMs; items in heavy-first order: dense heads and late query tiles
-// first).  A CTA runs one item at a time as a chain per key tile:
-// S = Q K^T -> softmax -> O += P V; the other CTA on the SM fills the tensor
-// core while this one is in its softmax.  Because each CTA's chain is
-// serial, one buffer each of Q, K and V (96 KB) hides the loads: K of tile
-// n+1 is fetched while tile n is in softmax and P V, V of tile n+1 while
-// tile n+1 is in S = Q K^T and softmax, and the next item's Q while the last
-// tile finishes.  A tcgen05.mma of M=128 with N >= 128 runs at the tensor
-// core's full rate; the issuing thread keeps its instruction stream between
-// MMAs to precomputed descriptor additions.
+// first).  Per CTA, tensor memory holds S (64 columns), two P buffers (bf16
+// pairs, 32 columns each) and O (128 columns): 256 columns, half an SM's.
+// Because S and P are separate, S = Q K^T of tile n+1 is issued as soon as
+// the softmax has read S of tile n, so the tensor core computes the next
+// scores while the softmax of the current tile runs; O += P V of tile n
+// follows the softmax.  The other CTA on the SM fills the remaining gaps.
 //
 // Roles (192 threads per CTA):
 //   warps 0-3  softmax: one thread per query row (warp w reads TMEM lanes
-//              32w..32w+31), all 128 key columns of the row.  Reads S from
-//              TMEM, masks, takes the row max, writes P = 2^(s - m) as bf16
-//              pairs over the first 64 columns of S, rescales O in TMEM only
-//              when the running max grew by more than 2^8, and after the
-//              item's last tile normalises O and stores the output rows.
-//   warp 4     one lane: TMA producer of Q, K and V;
-//   warp 5     allocates TMEM (256 columns: S/P at 0, O at 128) and one lane
-//              issues S = Q K^T (M=128, N=128, K=128; Q and K K-major in
-//              smem) and O += P V (M=128, N=128, K=128; P K-major in TMEM, V
-//              MN-major in smem) as tcgen05.mma with K=16 steps.
+//              32w..32w+31), all 64 key columns of the row.  Reads S, frees
+//              it, masks, takes the row max, writes P = 2^(s - m) as bf16 pairs
+//              into P buffer n%2, rescales O in TMEM only when the running max
+//              grew by more than 2^8, and after the item's last tile
+//              normalises O and stores the output rows.
+//   warp 4     one lane: TMA producer of Q (one buffer), K and V (two stages
+//              each);
+//   warp 5     allocates TMEM and one lane issues S = Q K^T (M=128, N=64,
+//              K=128; Q and K K-major in smem) and O += P V (M=128, N=128,
+//              K=64; P K-major in TMEM, V MN-major in smem) as tcgen05.mma with
+//              K=16 steps, from precomputed descriptors.  Per item: S(0), then
+//              S(j) and P V(j-1) for j >= 1, then P V of the last tile.
 // Every mbarrier wait is bounded; on expiry the CTA records RATP_ERR_TIMEOUT,
 // all roles drain out (copies and MMAs in flight are waited for), and TMEM
 // is released.
@@ -55,25 +54,28 @@ namespace ratp {
 namespace attn_tc {
 
 constexpr int BM = 128;          // queries per tile
-constexpr int BN = 128;          // keys per tile
+constexpr int BN = 64;           // keys per tile
 constexpr int DH = 128;          // head dim
 constexpr int kCtasPerSm = 2;
 constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 192;
-constexpr uint32_t kHalf = 128 * 64 * 2;       // 128 rows x 64 columns: 16 KB
-constexpr uint32_t kTile = 2 * kHalf;          // 128 x 128 bf16: 32 KB
+constexpr uint32_t kQHalf = BM * 64 * 2;       // Q: 128 rows x 64 columns: 16 KB
+constexpr uint32_t kQTile = 2 * kQHalf;        // 32 KB
+constexpr uint32_t kKHalf = BN * 64 * 2;       // K/V: 64 rows x 64 columns: 8 KB
+constexpr uint32_t kKTile = 2 * kKHalf;        // 16 KB
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kOffQ + kTile;
-constexpr uint32_t kOffV = kOffK + kTile;
-constexpr uint32_t kOffBar = kOffV + kTile;
-// barriers: qfull kfull vfull sfull pfull pvdone final
-constexpr uint32_t kNumBars = 7;
+constexpr uint32_t kOffK = kOffQ + kQTile;     // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kKTile; // 2 stages
+constexpr uint32_t kOffBar = kOffV + 2 * kKTile;
+// barriers: qfull qempty kfull[2] kempty[2] vfull[2] sfull sfree pfull[2] pvdone[2] final
+constexpr uint32_t kNumBars = 15;
 constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + TMEM slot, abort, alignment
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;      // S, then P over its first 64 columns
-constexpr uint32_t kColO = 128;    // O
+constexpr uint32_t kColS = 0;      // S: 64 columns
+constexpr uint32_t kColP = 64;     // P buffer b at 64 + 32 b
+constexpr uint32_t kColO = 128;    // O: 128 columns
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
@@ -83,6 +85,7 @@ struct Params {
   int n_dense, n_dil;
   int n_items_dense, n_items;
   float scale_log2;
+  int o_align32;          // output base 32-byte aligned (rows are 256 bytes)
   uint8_t dense_list[RATP_MAX_HEADS];
   uint8_t dil_list[RATP_MAX_HEADS];
 };
@@ -144,12 +147,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV;
   const uint32_t bar0 = sb + kOffBar;
   const uint32_t b_qfull = bar0 + 0 * 8;    // Q landed
-  const uint32_t b_kfull = bar0 + 1 * 8;    // K landed
-  const uint32_t b_vfull = bar0 + 2 * 8;    // V landed
-  const uint32_t b_sfull = bar0 + 3 * 8;    // S = Q K^T done (K and, at an item's end, Q free)
-  const uint32_t b_pfull = bar0 + 4 * 8;    // P written (128 softmax threads)
-  const uint32_t b_pvdone = bar0 + 5 * 8;   // O += P V done (V, S/P free; O current)
-  const uint32_t b_final = bar0 + 6 * 8;
+  const uint32_t b_qempty = bar0 + 1 * 8;   // last S = Q K^T of an item done
+  const uint32_t b_kfull = bar0 + 2 * 8;    // [2] K stage landed
+  const uint32_t b_kempty = bar0 + 4 * 8;   // [2] S = Q K^T read the K stage
+  const uint32_t b_vfull = bar0 + 6 * 8;    // [2] V stage landed
+  const uint32_t b_sfull = bar0 + 8 * 8;    // S = Q K^T done
+  const uint32_t b_sfree = bar0 + 9 * 8;    // S read by the softmax (128 threads)
+  const uint32_t b_pfull = bar0 + 10 * 8;   // [2] P buffer written (128 threads)
+  const uint32_t b_pvdone = bar0 + 12 * 8;  // [2] O += P V done: P buffer and V stage free
+  const uint32_t b_final = bar0 + 14 * 8;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 4);
 
@@ -158,11 +164,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
-    mbar_init(b_kfull, 1);
-    mbar_init(b_vfull, 1);
+    mbar_init(b_qempty, 1);
     mbar_init(b_sfull, 1);
-    mbar_init(b_pfull, kSoftmaxWarps * 32);
-    mbar_init(b_pvdone, 1);
+    mbar_init(b_sfree, kSoftmaxWarps * 32);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(b_kfull + 8 * i, 1);
+      mbar_init(b_kempty + 8 * i, 1);
+      mbar_init(b_vfull + 8 * i, 1);
+      mbar_init(b_pfull + 8 * i, kSoftmaxWarps * 32);
+      mbar_init(b_pvdone + 8 * i, 1);
+    }
     mbar_init(b_final, 1);
     *s_abort = 0;
     fence_barrier_init();
@@ -185,44 +196,48 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    // Tile n: Q (at an item's first tile) and K once S = Q K^T of tile n-1
-    // is done, V once O += P V of tile n-1 is done.
+    // Tile n (stage n%2): Q at an item's first tile once the previous item's
+    // last S = Q K^T is done; K once S = Q K^T of tile n-2 read the stage; V
+    // once O += P V of tile n-2 read the stage.
     if (lane == 0) {
-      int n = 0, nq = 0;                // tiles and Q loads issued
-      int last_k = -1, last_v = -1;     // tile of the last K / V load issued
+      int n = 0, li = 0;
+      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};   // last tile loaded per stage
       bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
         const Item it = make_item(p, idx);
+        if (li > 0 && !mbar_wait(b_qempty, (li - 1) & 1, s_abort)) { ok = false; break; }
+        mbar_arrive_expect_tx(b_qfull, kQTile);
+        tma_load_4d(sQ, &tm_q, b_qfull, 0, it.h, it.t0, it.b);
+        tma_load_4d(sQ + kQHalf, &tm_q, b_qfull, 64, it.h, it.t0, it.b);
         for (int j = 0; j < it.n_tiles; ++j, ++n) {
-          if (n > 0 && !mbar_wait(b_sfull, (n - 1) & 1, s_abort)) { ok = false; break; }
-          if (j == 0) {
-            mbar_arrive_expect_tx(b_qfull, kTile);
-            tma_load_4d(sQ, &tm_q, b_qfull, 0, it.h, it.t0, it.b);
-            tma_load_4d(sQ + kHalf, &tm_q, b_qfull, 64, it.h, it.t0, it.b);
-            ++nq;
-          }
+          const int st = n & 1;
           const bool pos = (j < it.n_win) || it.dense;
           const int row = (j < it.n_win) ? it.p_start + j * BN : (j - it.n_win) * BN;
+          if (n >= 2 && !mbar_wait(b_kempty + 8 * st, ((n - 2) >> 1) & 1, s_abort)) { ok = false; break; }
           if (!(blockIdx.x == 0 && (long long)n == g_fault_attn_ktile)) {   // else: planted failure
             const CUtensorMap* m = pos ? &tm_kpos : &tm_kdil;
-            mbar_arrive_expect_tx(b_kfull, kTile);
-            tma_load_4d(sK, m, b_kfull, 0, it.h, row, it.b);
-            tma_load_4d(sK + kHalf, m, b_kfull, 64, it.h, row, it.b);
-            last_k = n;
+            const uint32_t fb = b_kfull + 8 * st;
+            mbar_arrive_expect_tx(fb, kKTile);
+            tma_load_4d(sK + st * kKTile, m, fb, 0, it.h, row, it.b);
+            tma_load_4d(sK + st * kKTile + kKHalf, m, fb, 64, it.h, row, it.b);
+            last_k[st] = n;
           }
-          if (n > 0 && !mbar_wait(b_pvdone, (n - 1) & 1, s_abort)) { ok = false; break; }
+          if (n >= 2 && !mbar_wait(b_pvdone + 8 * st, ((n - 2) >> 1) & 1, s_abort)) { ok = false; break; }
           const CUtensorMap* m = pos ? &tm_vpos : &tm_vdil;
-          mbar_arrive_expect_tx(b_vfull, kTile);
-          tma_load_4d(sV, m, b_vfull, 0, it.h, row, it.b);
-          tma_load_4d(sV + kHalf, m, b_vfull, 64, it.h, row, it.b);
-          last_v = n;
+          const uint32_t fb = b_vfull + 8 * st;
+          mbar_arrive_expect_tx(fb, kKTile);
+          tma_load_4d(sV + st * kKTile, m, fb, 0, it.h, row, it.b);
+          tma_load_4d(sV + st * kKTile + kKHalf, m, fb, 64, it.h, row, it.b);
+          last_v[st] = n;
         }
       }
       // let the copies in flight land before the CTA ends (after an abort
-      // they may never have been consumed): the last Q, K and V load
-      if (nq > 0) mbar_drain(b_qfull, (nq - 1) & 1);
-      if (last_k >= 0) mbar_drain(b_kfull, last_k & 1);
-      if (last_v >= 0) mbar_drain(b_vfull, last_v & 1);
+      // they may never have been consumed)
+      if (li > 0) mbar_drain(b_qfull, (li - 1) & 1);
+      for (int st = 0; st < 2; ++st) {
+        if (last_k[st] >= 0) mbar_drain(b_kfull + 8 * st, (last_k[st] >> 1) & 1);
+        if (last_v[st] >= 0) mbar_drain(b_vfull + 8 * st, (last_v[st] >> 1) & 1);
+      }
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -231,34 +246,55 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       constexpr uint32_t idS = idesc_bf16_f32(BM, BN, 0, 0);    // Q K^T: both K-major
       constexpr uint32_t idPV = idesc_bf16_f32(BM, DH, 0, 1);   // P V: P K-major (TMEM), V MN-major
       const uint64_t dq = sw128_desc(sQ, 16, 1024);
-      const uint64_t dk = sw128_desc(sK, 16, 1024);
-      const uint64_t dv = sw128_desc(sV, kHalf, 1024);
-      const uint32_t tS = tmem + kColS, tO = tmem + kColO;
+      const uint64_t dk0 = sw128_desc(sK, 16, 1024);
+      const uint64_t dv0 = sw128_desc(sV, kKHalf, 1024);
+      constexpr uint64_t kStageDesc = kKTile >> 4;      // descriptor step between stages
+      const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO;
       int n = 0, li = 0;
       bool ok = true;
+      // S = Q K^T of tile n (its S columns were read by the softmax of n-1)
+      auto issue_s = [&](int nn) -> bool {
+        const int st = nn & 1;
+        if (nn > 0 && !mbar_wait(b_sfree, (nn - 1) & 1, s_abort)) return false;
+        if (!mbar_wait(b_kfull + 8 * st, (nn >> 1) & 1, s_abort)) return false;
+        tc_fence_after();
+        const uint64_t dk = dk0 + st * kStageDesc;
+#pragma unroll
+        for (int k = 0; k < DH / 16; ++k) {
+          const uint64_t oa = (uint64_t)(((k >> 2) * kQHalf + (k & 3) * 32) >> 4);
+          const uint64_t ob = (uint64_t)(((k >> 2) * kKHalf + (k & 3) * 32) >> 4);
+          umma_f16(tS, dq + oa, dk + ob, idS, k > 0 ? 1u : 0u);
+        }
+        umma_commit(b_sfull);
+        umma_commit(b_kempty + 8 * st);
+        return true;
+      };
+      // O += P V of tile nn (first = the item's first tile: O is overwritten)
+      auto issue_pv = [&](int nn, bool first) -> bool {
+        const int st = nn & 1;
+        if (!mbar_wait(b_pfull + 8 * st, (nn >> 1) & 1, s_abort)) return false;
+        if (!mbar_wait(b_vfull + 8 * st, (nn >> 1) & 1, s_abort)) return false;
+        tc_fence_after();
+        const uint64_t dv = dv0 + st * kStageDesc;
+        const uint32_t aP = tP + st * (BN / 2);
+        umma_f16_ts(tO, aP, dv, idPV, first ? 0u : 1u);
+#pragma unroll
+        for (int k = 1; k < BN / 16; ++k)
+          umma_f16_ts(tO, aP + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idPV, 1u);
+        umma_commit(b_pvdone + 8 * st);
+        return true;
+      };
       for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
         const int n_tiles = make_item(p, idx).n_tiles;
         if (!mbar_wait(b_qfull, li & 1, s_abort)) { ok = false; break; }
-        for (int j = 0; j < n_tiles; ++j, ++n) {
-          // S/P columns are free once O += P V of tile n-1 is done
-          if (n > 0 && !mbar_wait(b_pvdone, (n - 1) & 1, s_abort)) { ok = false; break; }
-          if (!mbar_wait(b_kfull, n & 1, s_abort)) { ok = false; break; }
-          tc_fence_after();
-#pragma unroll
-          for (int k = 0; k < DH / 16; ++k) {
-            const uint64_t off = (uint64_t)(((k >> 2) * kHalf + (k & 3) * 32) >> 4);
-            umma_f16(tS, dq + off, dk + off, idS, k > 0 ? 1u : 0u);
-          }
-          umma_commit(b_sfull);
-          if (!mbar_wait(b_pfull, n & 1, s_abort)) { ok = false; break; }
-          if (!mbar_wait(b_vfull, n & 1, s_abort)) { ok = false; break; }
-          tc_fence_after();
-          umma_f16_ts(tO, tS, dv, idPV, j > 0 ? 1u : 0u);
-#pragma unroll
-          for (int k = 1; k < BN / 16; ++k)
-            umma_f16_ts(tO, tS + k * 8, dv + (uint64_t)((k * 16 * 128) >> 4), idPV, 1u);
-          umma_commit(b_pvdone);
+        if (!issue_s(n)) { ok = false; break; }
+        for (int j = 1; j < n_tiles; ++j) {
+          if (!issue_s(n + j) || !issue_pv(n + j - 1, j == 1)) { ok = false; break; }
         }
+        if (!ok) break;
+        umma_commit(b_qempty);                       // all of this item's S = Q K^T issued
+        if (!issue_pv(n + n_tiles - 1, n_tiles == 1)) { ok = false; break; }
+        n += n_tiles;
       }
       // every MMA issued has completed before TMEM is released
       umma_commit(b_final);
@@ -269,7 +305,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     // ------------------------------------------------------------ softmax
     const int r = warp * 32 + lane;                  // query row within the tile (TMEM lane)
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const uint32_t colS = tl + kColS, colO = tl + kColO;
+    const uint32_t colS = tl + kColS, colP = tl + kColP, colO = tl + kColO;
     const float sc = p.scale_log2;
     // After a failed (timed-out or aborted) wait the warp leaves the loop;
     // every wait is warp-uniform, so warp-collective tcgen05 instructions are
@@ -283,13 +319,15 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int w_lo = max(t - p.W_eff + 1, 0);
       float m_used = -1e30f, l = 0.f;
       for (int j = 0; j < it.n_tiles; ++j, ++n) {
-        // S of tile n; its completion also covers O += P V of tile n-1
+        const int pb = n & 1;
         if (!warp_all(mbar_wait(b_sfull, n & 1, s_abort))) { ok = false; break; }
         tc_fence_after();
         uint32_t sr[BN];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(colS + 32 * c, sr + 32 * c);
+        tmem_ld32(colS, sr);
+        tmem_ld32(colS + 32, sr + 32);
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(b_sfree);                        // S may be overwritten now
 
         // valid columns [lo, hi) of this row in this tile, as 32-bit chunk masks
         int lo, hi;
@@ -301,9 +339,9 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           lo = 0;
           hi = lim_dil - (j - it.n_win) * BN;
         }
-        uint32_t vm[4];
+        uint32_t vm[2];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           const int clo = min(max(lo - 32 * c, 0), 32);
           const int chi = min(max(hi - 32 * c, 0), 32);
           vm[c] = (chi >= 32 ? 0xffffffffu : ((1u << chi) - 1u)) & ~(clo >= 32 ? 0xffffffffu : ((1u << clo) - 1u));
@@ -311,7 +349,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         // mask in place (invalid -> -inf), then the row max of raw scores
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           if (!__all_sync(0xffffffffu, vm[c] == 0xffffffffu)) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
@@ -344,16 +382,16 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           l *= alpha;
           m_used = mxs;
         }
-        // p = 2^(s*scale - m) as bf16 pairs over S columns 16c..16c+15
+        // p = 2^(s*scale - m) as bf16 pairs
         const float2 sc2 = make_float2(sc, sc);
         const float2 nm2 = make_float2(-m_used, -m_used);
         float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        uint32_t w[BN / 2];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t w[16];
+        for (int c = 0; c < 2; ++c) {
           if (__all_sync(0xffffffffu, vm[c] == 0u)) {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) w[i] = 0u;
+            for (int i = 0; i < 16; ++i) w[16 * c + i] = 0u;
           } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -361,13 +399,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                 __uint_as_float(sr[32 * c + 2 * i + 1])), sc2, nm2);
               const float2 e = make_float2(exp2f(x.x), exp2f(x.y));
               ls[i & 1] = add2(ls[i & 1], e);
-              w[i] = pack_bf16x2(e.x, e.y);
+              w[16 * c + i] = pack_bf16x2(e.x, e.y);
             }
           }
-          tmem_st16(colS + 16 * c, w);
         }
         l += (ls[0].x + ls[0].y) + (ls[1].x + ls[1].y);
+        // P buffer pb was last read by O += P V of tile n-2
+        if (n >= 2 && !warp_all(mbar_wait(b_pvdone + 8 * pb, ((n - 2) >> 1) & 1, s_abort))) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32(colP + pb * (BN / 2), w);
         if (rescale) {
+          // O must hold P V of tile n-1 before it is scaled
+          if (!warp_all(mbar_wait(b_pvdone + 8 * (pb ^ 1), ((n - 1) >> 1) & 1, s_abort))) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t o32[32];
@@ -380,11 +424,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(b_pfull);
+        mbar_arrive(b_pfull + 8 * pb);
       }
       if (!ok) break;
       // epilogue: wait for the item's last P V, normalise, store
-      if (!warp_all(mbar_wait(b_pvdone, (n - 1) & 1, s_abort))) { ok = false; break; }
+      const int nl = n - 1;
+      if (!warp_all(mbar_wait(b_pvdone + 8 * (nl & 1), (nl >> 1) & 1, s_abort))) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.f / l;
       __nv_bfloat16* orow = p.o + (((size_t)it.b * p.T + t) * p.H + it.h) * DH;
@@ -395,13 +440,19 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         tmem_wait_ld();
         if (t < p.T) {
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 pk;
-            pk.x = pack_bf16x2(__uint_as_float(o32[8 * v + 0]) * inv, __uint_as_float(o32[8 * v + 1]) * inv);
-            pk.y = pack_bf16x2(__uint_as_float(o32[8 * v + 2]) * inv, __uint_as_float(o32[8 * v + 3]) * inv);
-            pk.z = pack_bf16x2(__uint_as_float(o32[8 * v + 4]) * inv, __uint_as_float(o32[8 * v + 5]) * inv);
-            pk.w = pack_bf16x2(__uint_as_float(o32[8 * v + 6]) * inv, __uint_as_float(o32[8 * v + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * v) = pk;
+          for (int v = 0; v < 2; ++v) {
+            uint32_t q[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              q[i] = pack_bf16x2(__uint_as_float(o32[16 * v + 2 * i]) * inv, __uint_as_float(o32[16 * v + 2 * i + 1]) * inv);
+            if (p.o_align32) {                       // one 32-byte store per 16 values
+              asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                           :: "l"(orow + 32 * c + 16 * v), "r"(q[0]), "r"(q[1]), "r"(q[2]), "r"(q[3]),
+                              "r"(q[4]), "r"(q[5]), "r"(q[6]), "r"(q[7]) : "memory");
+            } else {                                 // output only 16-byte aligned
+              *reinterpret_cast<uint4*>(orow + 32 * c + 16 * v) = make_uint4(q[0], q[1], q[2], q[3]);
+              *reinterpret_cast<uint4*>(orow + 32 * c + 16 * v + 8) = make_uint4(q[4], q[5], q[6], q[7]);
+            }
           }
         }
       }

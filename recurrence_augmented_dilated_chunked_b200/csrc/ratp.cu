@@ -265,6 +265,7 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
   p.n_items_dense = B * p.n_dense * p.NQ;
   p.n_items = B * H * p.NQ;
   p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
+  p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   const long long row = (long long)H * 128, bat = (long long)T * row;
   CUtensorMap tq, tkp, tvp, tkd, tvd;
   constexpr int qr = attn_tc::BM, kr = attn_tc::BN;

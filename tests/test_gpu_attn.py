@@ -57,6 +57,22 @@ def test_tensor_core_attention_matches_oracle(B, T, H, D, W, dense, qs):
     assert_close(o, ref, "bf16", "tc attention")
 
 
+def test_tensor_core_attention_output_only_16_byte_aligned():
+    """An output view that starts 16 bytes into its buffer takes the 16-byte
+    store path of the epilogue and gives the same values."""
+    B, T, H, D, W = 1, 300, 2, 8, 16
+    q, k, v = _qkv(B, T, H, 128, "bf16", seed=5)
+    buf = torch.empty(B * T * H * 128 + 8, dtype=torch.bfloat16, device=DEV)
+    o = buf[8:].view(B, T, H, 128)
+    assert o.data_ptr() % 32 == 16
+    ratp.dilated_attn_prefill(q.to(DEV), k.to(DEV), v.to(DEV), D, W, out=o)
+    ratp.last_error()
+    ref = oracle.attention(to64(q), to64(k), to64(v), D, W)
+    assert_close(o, ref, "bf16", "tc attention, 16-byte aligned output")
+    o2 = ratp.dilated_attn_prefill(q.to(DEV), k.to(DEV), v.to(DEV), D, W)
+    assert bits_equal(o2, o)
+
+
 SIMT_CASES = [
     ("f32", 64, 1, 256, 2, 4, 0, ()),        # the fp32 parity workload, full size
     ("f32", 64, 2, 300, 3, 3, 5, (1,)),
