@@ -276,6 +276,90 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- GPU arm
+OTHER_CONFIGS = ["bf16_1p5b_T4096_D16", "bf16_hybrid_7p6b_T8192_D4"]
+
+
+def measure_config(name, dev, steps, warmup, peaks):
+    """Prefill (and, where the workload has them, decode steps continuing from
+    the prefill) of one more configuration, timed with CUDA events on the
+    launching stream.  Reported beside the headline line, not part of it."""
+    import recurrence_augmented_dilated_chunked_b200 as ratp
+    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, decode_inputs, prefill_inputs
+    w = WORKLOADS[name]
+    stream = torch.cuda.current_stream(dev)
+    q, xk, xv, g = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.H, w.Dh, w.dtype,
+                                                        w.gate_mean, w.gate_std, seed=0))
+    hk, hv, o = (torch.empty_like(q) for _ in range(3))
+    fs = torch.empty(2, w.B, w.H, w.Dh, dtype=torch.float32, device=dev)
+    ws = ratp.scan_workspace(w.B, w.T, w.H, w.Dh, q.dtype, dev)
+    mask = w.dense_mask if w.dense_heads else None
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(warmup + steps):
+        ev = evs[i - warmup] if i >= warmup else None
+        if ev:
+            ev[0].record(stream)
+        ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, final_state=fs, workspace=ws)
+        if ev:
+            ev[1].record(stream)
+        ratp.dilated_attn_prefill(q, hk, hv, w.D, w.W, head_mask=mask, out=o)
+        if ev:
+            ev[2].record(stream)
+    torch.cuda.synchronize()
+    ratp.last_error(dev)
+    scan_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    pc = prefill_counts(w)
+    scan_gbs = pc["scan_bytes"] / (scan_ms / 1e3) / 1e9
+    attn_gbs = pc["attn_bytes"] / (attn_ms / 1e3) / 1e9
+    attn_tfs = pc["attn_flops"] / (attn_ms / 1e3) / 1e12
+    out = {"B": w.B, "T": w.T, "H": w.H, "Dh": w.Dh, "D": w.D, "W": w.W,
+           "dense_heads": list(w.dense_heads),
+           "prefill_tokens_per_s": w.B * w.T / ((scan_ms + attn_ms) / 1e3),
+           "scan_ms": scan_ms, "scan_frac_hbm": scan_gbs / peaks["hbm_gbs"],
+           "attn_ms": attn_ms, "attn_frac_hbm": attn_gbs / peaks["hbm_gbs"],
+           "attn_tflops": attn_tfs, "attn_frac_tensor": attn_tfs / peaks["bf16_tflops"],
+           "attn_pairs": pc["pairs"], "attn_flops": pc["attn_flops"]}
+    del xk, xv, g, ws
+    if w.decode_steps:
+        n = w.decode_steps
+        cache = ratp.KVCache(w.B, w.H, w.Dh, w.T + n, w.D, w.W, head_mask=mask, device=dev)
+        cache.pack(hk, hv, w.T)
+        lens = cache.lengths()
+        dq, dxk, dxv, dg = (t.to(dev) for t in decode_inputs(n, w.B, w.H, w.Dh, w.dtype,
+                                                              w.gate_mean, w.gate_std))
+        state = fs.clone()
+        dout = torch.empty(n, w.B, w.H, w.Dh, dtype=torch.bfloat16, device=dev)
+
+        def burst():
+            lens.fill_(w.T)
+            state.copy_(fs)
+            for i in range(n):
+                cache.decode_step(dq[i], dxk[i], dxv[i], dg[i], state, out=dout[i])
+
+        burst()
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            burst()
+        for _ in range(warmup):
+            graph.replay()
+        d_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for e in d_evs:
+            e[0].record(stream)
+            graph.replay()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        ratp.last_error(dev)
+        dec_ms = statistics.median(e[0].elapsed_time(e[1]) for e in d_evs) / n
+        dec_bytes = sum(decode_bytes_per_step(w, w.T + i) for i in range(n)) / n
+        dec_gbs = dec_bytes / (dec_ms / 1e3) / 1e9
+        out.update({"decode_steps": n, "decode_tokens_per_s": w.B / (dec_ms / 1e3),
+                    "decode_ms_per_step": dec_ms, "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
+                    "decode_alg_bytes_per_step": dec_bytes})
+        del graph
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import recurrence_augmented_dilated_chunked_b200 as ratp
     from recurrence_augmented_dilated_chunked_b200 import (WORKLOADS, decode_context,
@@ -457,6 +541,10 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk.summary(),
         "wall_s": t_wall,
     }
+    if not args.no_other_configs:
+        # the other workloads, measured after the timed region (not part of it)
+        line["other_configs"] = {n: measure_config(n, dev, min(args.steps, 5), args.warmup, peaks)
+                                 for n in OTHER_CONFIGS}
     if not args.no_cpu_baseline and world >= 1:
         line["cpu_baseline"] = oracle_sample()
     print(json.dumps(line), flush=True)
@@ -471,6 +559,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the per-configuration measurements of the other workloads")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run only this part, untimed (a driver for ncu captures)")
     args = ap.parse_args()
