@@ -4,7 +4,7 @@
 // section 6: dense heads).
 //
 // Decode step for token t = len[b] of every sequence, one launch:
-//   grid (split, h, b).  The keys of (b, h) form a virtual list: the cached
+//   grid: one CTA per (b, h, split).  The keys of (b, h) form a virtual list: the cached
 //   dilated slots whose positions lie before the window, s < (t-W+1) / D_h
 //   (all s < t / D_h without a window; Kc/Vc rows), then every window position
 //   t-W < p < t (ring rows), so each key appears once.  Split i streams keys
@@ -43,6 +43,8 @@ struct Params {
   long long rows_per_b;
   int B, H, D, W, T_max, split_keys, max_splits;
   float scale_log2;
+  int splits_per_b;             // CTAs per batch item: sum over heads of split_base
+  int split_base[RATP_MAX_HEADS + 1];   // first CTA (within a batch item) of each head
   unsigned long long dense_bits[RATP_MAX_HEADS / 64];
 };
 
@@ -72,7 +74,26 @@ decode_kernel(const Params p) {
   __shared__ float s_acc[NG][DH];
   __shared__ int s_last;
 
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream: let the next step be scheduled now, then wait until everything
+  // before this step has completed and is visible.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // 1-D grid: batch item, then head (each head gets the splits its largest
+  // key count can need), then split
+  const int b = blockIdx.x / p.splits_per_b;
+  const int rem = blockIdx.x - b * p.splits_per_b;
+  int h = 0;
+  {
+    int lo = 0, hi = p.H - 1;                    // last head with split_base[h] <= rem
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (p.split_base[mid] <= rem) lo = mid; else hi = mid - 1;
+    }
+    h = lo;
+  }
+  const int split = rem - p.split_base[h];
   const int tid = threadIdx.x;
   const int t = p.len[b];
   const bool dense = is_dense(p.dense_bits, h);
@@ -258,7 +279,7 @@ decode_kernel(const Params p) {
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    const unsigned int total = gridDim.x * gridDim.y * gridDim.z;
+    const unsigned int total = gridDim.x;
     const unsigned int prev = atomicAdd(p.counters + (long long)p.B * p.H, 1u);
     if (prev == total - 1) {
       __threadfence();

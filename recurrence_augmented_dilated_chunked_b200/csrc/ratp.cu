@@ -598,9 +598,35 @@ int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* 
   int rc = read_mask(c->dense, c->H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
   if (rc) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  dim3 grid((unsigned)c->max_splits, (unsigned)c->H, (unsigned)c->B);
-  if (c->Dh == 128) decode::decode_kernel<128><<<grid, decode::kThreads, 0, st>>>(p);
-  else decode::decode_kernel<64><<<grid, decode::kThreads, 0, st>>>(p);
+  // per-head split counts: the most keys head h can hold, over split_keys
+  p.split_base[0] = 0;
+  for (int h = 0; h < c->H; ++h) {
+    const bool dense = (p.dense_bits[h >> 6] >> (h & 63)) & 1ull;
+    const long long keys = dense ? (long long)c->T_max : (long long)c->T_max / c->D + c->W;
+    long long sp = (keys + c->split_keys - 1) / c->split_keys;
+    if (sp < 1) sp = 1;
+    if (sp > c->max_splits) sp = c->max_splits;
+    p.split_base[h + 1] = p.split_base[h] + (int)sp;
+  }
+  p.splits_per_b = p.split_base[c->H];
+  if ((long long)p.splits_per_b * c->B > 0x7fffffffll) return RATP_ERR_SHAPE;
+  dim3 grid((unsigned)(p.splits_per_b * c->B));
+  // Programmatic dependent launch: the step may be scheduled while the
+  // previous kernel in the stream drains; it waits for that kernel's
+  // completion (griddepcontrol.wait) before touching any memory.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(decode::kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = (c->Dh == 128) ? cudaLaunchKernelEx(&cfg, decode::decode_kernel<128>, p)
+                                 : cudaLaunchKernelEx(&cfg, decode::decode_kernel<64>, p);
+  if (e != cudaSuccess) return RATP_ERR_CUDA;
   return launch_status();
 }
 
