@@ -196,19 +196,17 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
-    // Tile n (stage n%2): Q at an item's first tile once the previous item's
-    // last S = Q K^T is done; K once S = Q K^T of tile n-2 read the stage; V
-    // once O += P V of tile n-2 read the stage.
+    // Tile n (stage n%2): K once S = Q K^T of tile n-2 read the stage; at an
+    // item's first tile then Q, once the previous item's last S = Q K^T is
+    // done (its K load is already under way); V once O += P V of tile n-2
+    // read the stage.  The next item's Q is prefetched into L2 one item
+    // ahead, so its load at the item boundary is an L2 hit.
     if (lane == 0) {
-      int n = 0, li = 0;
+      int n = 0, li = 0, nq = 0;
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};   // last tile loaded per stage
       bool ok = true;
       for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
         const Item it = make_item(p, idx);
-        if (li > 0 && !mbar_wait(b_qempty, (li - 1) & 1, s_abort)) { ok = false; break; }
-        mbar_arrive_expect_tx(b_qfull, kQTile);
-        tma_load_4d(sQ, &tm_q, b_qfull, 0, it.h, it.t0, it.b);
-        tma_load_4d(sQ + kQHalf, &tm_q, b_qfull, 64, it.h, it.t0, it.b);
         for (int j = 0; j < it.n_tiles; ++j, ++n) {
           const int st = n & 1;
           const bool pos = (j < it.n_win) || it.dense;
@@ -222,6 +220,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             tma_load_4d(sK + st * kKTile + kKHalf, m, fb, 64, it.h, row, it.b);
             last_k[st] = n;
           }
+          if (j == 0) {
+            if (li > 0 && !mbar_wait(b_qempty, (li - 1) & 1, s_abort)) { ok = false; break; }
+            mbar_arrive_expect_tx(b_qfull, kQTile);
+            tma_load_4d(sQ, &tm_q, b_qfull, 0, it.h, it.t0, it.b);
+            tma_load_4d(sQ + kQHalf, &tm_q, b_qfull, 64, it.h, it.t0, it.b);
+            ++nq;
+          }
           if (n >= 2 && !mbar_wait(b_pvdone + 8 * st, ((n - 2) >> 1) & 1, s_abort)) { ok = false; break; }
           const CUtensorMap* m = pos ? &tm_vpos : &tm_vdil;
           const uint32_t fb = b_vfull + 8 * st;
@@ -233,7 +238,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       // let the copies in flight land before the CTA ends (after an abort
       // they may never have been consumed)
-      if (li > 0) mbar_drain(b_qfull, (li - 1) & 1);
+      if (nq > 0) mbar_drain(b_qfull, (nq - 1) & 1);
       for (int st = 0; st < 2; ++st) {
         if (last_k[st] >= 0) mbar_drain(b_kfull + 8 * st, (last_k[st] >> 1) & 1);
         if (last_v[st] >= 0) mbar_drain(b_vfull + 8 * st, (last_v[st] >> 1) & 1);

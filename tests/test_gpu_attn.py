@@ -153,3 +153,12 @@ def test_full_size_end_to_end_sampled_rows(name):
     o_cpu = o.cpu()
     got = torch.stack([o_cpu[b, t, heads[hi]] for b, t, hi in rows])
     assert_close(got, ref, "bf16", name)
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 0, 2), (0, 16, 2), (2, 16, 0)])
+def test_empty_problem_launches_nothing(B, T, H):
+    """An empty batch, sequence or head set is a no-op that succeeds."""
+    q = torch.empty(B, T, H, 128, dtype=torch.bfloat16, device=DEV)
+    o = ratp.dilated_attn_prefill(q, q, q, 4, 8)
+    ratp.last_error()
+    assert o.shape == q.shape

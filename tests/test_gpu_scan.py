@@ -90,3 +90,11 @@ def test_scan_full_size_sampled_channels(name):
     assert_close(hk.reshape(w.B, w.T, C)[:, :, cols], rk, w.dtype, "hk sampled")
     assert_close(hv.reshape(w.B, w.T, C)[:, :, cols], rv, w.dtype, "hv sampled")
     assert_close(fs[0].reshape(w.B, C)[:, cols], rk[:, -1], "f32", "final state sampled")
+
+
+@pytest.mark.parametrize("B,T", [(1, 0), (0, 32)])
+def test_scan_empty_sequence_is_a_no_op(B, T):
+    x = torch.empty(B, T, 2, 64, dtype=torch.bfloat16, device=DEV)
+    hk, hv = ratp.scan_prefill_kv(x, x, x)
+    ratp.last_error()
+    assert hk.shape == x.shape and hv.shape == x.shape
