@@ -44,6 +44,8 @@ TC_CASES = [
     (2, 700, 4, 4, 0, (0, 1), 4.0),
     (1, 1100, 2, 64, 128, (1,), 3.0),
     (1, 2049, 1, 16, 200, (), 2.0),
+    # the most heads a launch takes, every seventh one dense
+    (1, 130, 256, 2, 3, tuple(range(0, 256, 7)), 1.0),
 ]
 
 

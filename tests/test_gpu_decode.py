@@ -27,15 +27,15 @@ def _dil(h, D, mask):
     return 1 if (mask and mask[h]) else D
 
 
-@pytest.mark.parametrize("B,T,n,H,D,W,dense", [
-    (2, 200, 70, 4, 4, 0, (0,)),
-    (2, 131, 40, 2, 16, 16, ()),
-    (1, 5, 30, 2, 3, 8, (1,)),
-    (3, 300, 20, 2, 64, 128, ()),
-    (1, 1, 10, 1, 1, 0, ()),
+@pytest.mark.parametrize("B,T,n,H,D,W,dense,Dh", [
+    (2, 200, 70, 4, 4, 0, (0,), 128),
+    (2, 131, 40, 2, 16, 16, (), 128),
+    (1, 5, 30, 2, 3, 8, (1,), 128),
+    (3, 300, 20, 2, 64, 128, (), 128),
+    (1, 1, 10, 1, 1, 0, (), 128),
+    (2, 100, 25, 3, 4, 8, (1,), 64),
 ])
-def test_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, dense):
-    Dh = 128
+def test_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, dense, Dh):
     mask = [1 if h in dense else 0 for h in range(H)]
     N = T + n
     q, xk, xv, g = prefill_inputs(B, N, H, Dh, "bf16", gate_mean=1.0, gate_std=2.0, seed=N)

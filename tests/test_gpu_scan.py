@@ -11,9 +11,11 @@ from parity import assert_close, bits_equal, to64
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
-# T spans several chunks (128 tokens for bf16, 64 for fp32) and ragged tails.
+# T spans several chunks (256 tokens for bf16, 128 for fp32) and ragged tails;
+# the largest case has 4096 channels per token (64 slabs of 64).
 SHAPES = [(1, 1, 1, 64), (2, 5, 1, 64), (1, 63, 2, 64), (1, 64, 1, 64), (2, 127, 1, 128),
-          (1, 128, 1, 64), (1, 129, 2, 64), (3, 1000, 2, 64), (1, 4099, 4, 128), (2, 8191, 1, 64)]
+          (1, 128, 1, 64), (1, 129, 2, 64), (1, 255, 1, 64), (1, 256, 2, 64), (2, 257, 1, 128),
+          (3, 1000, 2, 64), (1, 4099, 4, 128), (2, 8191, 1, 64), (1, 300, 32, 128)]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
