@@ -16,7 +16,7 @@
 //   (the query's own key).  None of these rows is read by any CTA of the
 //   same step, so there is no intra-step race.
 //   Splits publish (m, l, acc) partials; the last split of (b, h) to finish
-//   (atomic counter) merges them and writes o.  The last CTA of the grid
+//   (atomic counter) merges them and writes o.  The last CTA of batch item b
 //   advances len[b].  Counters return to zero, so no per-step reset is needed.
 #pragma once
 #include "common.cuh"
@@ -39,7 +39,7 @@ struct Params {
   __nv_bfloat16* Vw;
   int32_t* len;
   float* partial;               // [B][H][max_splits][Dh + 2]
-  uint32_t* counters;           // [B*H + 1]
+  uint32_t* counters;           // [B*H] per (b, h), then [B] per batch item
   long long rows_per_b;
   int B, H, D, W, T_max, split_keys, max_splits;
   float scale_log2;
@@ -275,19 +275,19 @@ decode_kernel(const Params p) {
     }
   }
 
-  // ---- the last CTA of the grid advances len ----
+  // ---- the last CTA of batch item b advances len[b] ----
+  // (one counter per batch item, so the step's closing atomics spread over
+  // B addresses instead of one)
   __syncthreads();
   if (tid == 0) {
     __threadfence();
-    const unsigned int total = gridDim.x;
-    const unsigned int prev = atomicAdd(p.counters + (long long)p.B * p.H, 1u);
-    if (prev == total - 1) {
+    uint32_t* cnt = p.counters + (long long)p.B * p.H + b;
+    const unsigned int prev = atomicAdd(cnt, 1u);
+    if (prev == (unsigned int)p.splits_per_b - 1u) {
       __threadfence();
-      for (int bb = 0; bb < p.B; ++bb) {
-        const int tb = p.len[bb];
-        if (tb < p.T_max) p.len[bb] = tb + 1;
-      }
-      p.counters[(long long)p.B * p.H] = 0u;
+      const int tb = p.len[b];
+      if (tb < p.T_max) p.len[b] = tb + 1;
+      *cnt = 0u;
       __threadfence();
     }
   }

@@ -332,7 +332,7 @@ int cache_layout(int B, int H, int Dh, int T_max, int D, int W, const uint8_t* h
   L->off_vw = take((size_t)B * H * W * row_bytes);
   L->off_len = take((size_t)B * 4);
   L->off_part = take((size_t)B * H * L->max_splits * (Dh + 2) * 4);
-  L->off_cnt = take((size_t)(B * H + 1) * 4);
+  L->off_cnt = take((size_t)(B * H + B) * 4);
   L->total = off;
   return RATP_OK;
 }
@@ -533,7 +533,7 @@ int ratp_cache_init(ratp_cache* c, void* buffer, size_t bytes, int B, int H, int
   for (int h = 0; h < H; ++h) c->dense[h] = (head_mask != nullptr && head_mask[h] != 0) ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(c->len, 0, (size_t)B * 4, st) != cudaSuccess) return RATP_ERR_CUDA;
-  if (cudaMemsetAsync(c->counters, 0, (size_t)(B * H + 1) * 4, st) != cudaSuccess) return RATP_ERR_CUDA;
+  if (cudaMemsetAsync(c->counters, 0, (size_t)(B * H + B) * 4, st) != cudaSuccess) return RATP_ERR_CUDA;
   return RATP_OK;
 }
 
