@@ -62,7 +62,7 @@ __device__ __forceinline__ long long head_offset(const unsigned long long* bits,
 }
 
 template <int DH>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 7)
 decode_kernel(const Params p) {
   constexpr int LPK = DH / 8;                    // lanes per key (8 bf16 per lane)
   constexpr int KPW = 32 / LPK;                  // keys per warp per step
@@ -185,6 +185,9 @@ decode_kernel(const Params p) {
           }
         }
       }
+      // scores of the block's keys, then one max and one rescale per block
+      float sc_[UNROLL];
+      float m_blk = m;
 #pragma unroll
       for (int u = 0; u < UNROLL; ++u) {
         float kf[8];
@@ -194,16 +197,25 @@ decode_kernel(const Params p) {
         for (int i = 0; i < 8; ++i) s = fmaf(qf[i], kf[i], s);
 #pragma unroll
         for (int off = LPK / 2; off > 0; off >>= 1) s += __shfl_xor_sync(sub_mask, s, off, LPK);
-        if (use[u]) {
-          float vf[8];
-          Elem<__nv_bfloat16>::unpack(vv[u], vf);
-          const float m_new = fmaxf(m, s);
-          const float alpha = exp2f(m - m_new);
-          const float pj = exp2f(s - m_new);
-          l = l * alpha + pj;
+        sc_[u] = use[u] ? s : -INFINITY;
+        m_blk = fmaxf(m_blk, sc_[u]);
+      }
+      if (m_blk != -INFINITY) {
+        const float alpha = exp2f(m - m_blk);      // m = -inf on the first block: alpha = 0
+        l *= alpha;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(acc[i], alpha, pj * vf[i]);
-          m = m_new;
+        for (int i = 0; i < 8; ++i) acc[i] *= alpha;
+        m = m_blk;
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u) {
+          if (use[u]) {
+            float vf[8];
+            Elem<__nv_bfloat16>::unpack(vv[u], vf);
+            const float pj = exp2f(sc_[u] - m);
+            l += pj;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = fmaf(pj, vf[i], acc[i]);
+          }
         }
       }
     }
