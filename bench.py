@@ -53,12 +53,13 @@ def attention_pairs(T, D, W, dense=False):
 
 def prefill_counts(w):
     E = w.B * w.T * w.H * w.Dh
+    esz = 4 if w.dtype == "f32" else 2
     pairs = 0
     for h in range(w.H):
         pairs += w.B * attention_pairs(w.T, w.D, w.W, dense=h in w.dense_heads)
     return {
-        "scan_bytes": 5 * E * 2,                  # read xk, xv, g; write hk, hv (bf16)
-        "attn_bytes": 4 * E * 2,                  # read q, hk, hv; write o
+        "scan_bytes": 5 * E * esz,                # read xk, xv, g; write hk, hv
+        "attn_bytes": 4 * E * esz,                # read q, hk, hv; write o
         "attn_flops": 4 * w.Dh * pairs,           # QK^T + PV over the key sets
         "pairs": pairs,
     }
@@ -276,7 +277,8 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- GPU arm
-OTHER_CONFIGS = ["bf16_1p5b_T4096_D16", "bf16_hybrid_7p6b_T8192_D4"]
+# the fp32 workload is a parity configuration: its line is latency, not a roofline
+OTHER_CONFIGS = ["bf16_1p5b_T4096_D16", "bf16_hybrid_7p6b_T8192_D4", "f32_small_T256_D4"]
 
 
 def measure_config(name, dev, steps, warmup, peaks):
