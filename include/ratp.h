@@ -105,8 +105,8 @@ int ratp_debug_fault(int kind, long long arg);
  * workspace: device scratch of at least ratp_scan_workspace_bytes.  It must
  *   be zero-filled once before its first use; every call leaves it valid for
  *   the next one (each launch tags its chunk descriptors with a fresh launch
- *   number), and calls sharing one workspace must be ordered on one stream.  h may alias x (in-place) only when
- *   T == 1.  Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of
+ *   number), and calls sharing one workspace must be ordered on one stream.
+ *   h may alias x (in-place) only when T == 1.  Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of
  *   64), ALIGN, CAPACITY (workspace too small).  T == 0 or B == 0 is a no-op.
  * ---------------------------------------------------------------------- */
 int ratp_scan_workspace_bytes(int B, int T, int H, int Dh, int dtype, size_t* bytes);
@@ -201,7 +201,7 @@ typedef struct ratp_cache {
   int64_t rows_per_b;   /* sum_h cap_h */
   int32_t B, H, Dh, T_max, D, W;
   int32_t split_keys;   /* keys per decode split */
-  int32_t max_splits;   /* grid width of one decode step */
+  int32_t max_splits;   /* most decode splits any head can need (partial rows per (b, h)) */
   uint8_t dense[RATP_MAX_HEADS];
 } ratp_cache;
 
