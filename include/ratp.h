@@ -106,8 +106,9 @@ int ratp_debug_fault(int kind, long long arg);
  *   be zero-filled once before its first use; every call leaves it valid for
  *   the next one (each launch tags its chunk descriptors with a fresh launch
  *   number), and calls sharing one workspace must be ordered on one stream.
- *   h may alias x (in-place) only when T == 1.  Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of
- *   64), ALIGN, CAPACITY (workspace too small).  T == 0 or B == 0 is a no-op.
+ *   h may alias x (in-place) only when T == 1.
+ * Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of 64), ALIGN,
+ *   CAPACITY (workspace too small).  T == 0 or B == 0 is a no-op.
  * ---------------------------------------------------------------------- */
 int ratp_scan_workspace_bytes(int B, int T, int H, int Dh, int dtype, size_t* bytes);
 int ratp_scan_prefill(const void* x, const void* g, void* h, float* final_state,
