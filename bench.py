@@ -372,6 +372,21 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     wp, wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
 
+    if args.only == "prefill":
+        # profiling driver: prefill passes of one workload, no timing or report
+        w = WORKLOADS[args.workload or PREFILL]
+        q, xk, xv, g = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.H, w.Dh, w.dtype,
+                                                            w.gate_mean, w.gate_std, seed=rank))
+        hk, hv, o = (torch.empty_like(q) for _ in range(3))
+        ws = ratp.scan_workspace(w.B, w.T, w.H, w.Dh, q.dtype, dev)
+        mask = w.dense_mask if w.dense_heads else None
+        for _ in range(args.warmup + args.steps):
+            ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, workspace=ws)
+            ratp.dilated_attn_prefill(q, hk, hv, w.D, w.W, head_mask=mask, out=o)
+        torch.cuda.synchronize()
+        ratp.last_error(dev)
+        return 0
+
     # ---- prefill inputs (seeded, synthetic; a different seed per rank) ----
     q, xk, xv, g = prefill_inputs(wp.B, wp.T, wp.H, wp.Dh, wp.dtype, wp.gate_mean, wp.gate_std,
                                   seed=rank)
@@ -415,14 +430,6 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     ratp.last_error(dev)
 
-    if args.only == "prefill":
-        # profiling driver: prefill passes only, no timing or report
-        for _ in range(args.warmup + args.steps):
-            ratp.scan_prefill_kv(xkd, xvd, gd, hk=hk, hv=hv, workspace=ws)
-            ratp.dilated_attn_prefill(qd, hk, hv, wp.D, wp.W, out=o)
-        torch.cuda.synchronize()
-        ratp.last_error(dev)
-        return 0
     if args.only == "decode":
         # profiling driver: decode bursts only (graph replays), no report
         for _ in range(args.warmup + args.steps):
@@ -604,6 +611,8 @@ def main():
                     help="skip the per-configuration measurements of the other workloads")
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="run only this part, untimed (a driver for ncu captures)")
+    ap.add_argument("--workload", default=None,
+                    help="with --only prefill: the prefill workload (default: the headline one)")
     args = ap.parse_args()
     if args.warmup < 3 and args.only is None:
         ap.error("--warmup must be >= 3")
