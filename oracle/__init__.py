@@ -54,6 +54,7 @@ def _load():
     if _lib is None:
         lib = ctypes.CDLL(build())
         lib.orc_scan.argtypes = [_D, _D, _D, ctypes.c_long, ctypes.c_long, ctypes.c_long]
+        lib.orc_scan_reset.argtypes = [_D, _D, _D] + [ctypes.c_long] * 4
         lib.orc_scan_step.argtypes = [_D, _D, _D, ctypes.c_long]
         lib.orc_key_set.argtypes = [ctypes.c_long, ctypes.c_long, ctypes.c_long, _L]
         lib.orc_key_set.restype = ctypes.c_long
@@ -66,7 +67,7 @@ def _load():
         lib.orc_ring_row.argtypes = [ctypes.c_long] * 5
         lib.orc_ring_row.restype = ctypes.c_long
         lib.orc_cache_pack.argtypes = [_D, _D] + [ctypes.c_long] * 7 + [_U8, _D, _D, _D, _D, _L]
-        lib.orc_decode_step.argtypes = [_D] * 9 + [_L, _D] + [ctypes.c_long] * 6 + [_U8]
+        lib.orc_decode_step.argtypes = [_D] * 9 + [_L, _D] + [ctypes.c_long] * 6 + [_U8, ctypes.c_long]
         lib.orc_decode_step.restype = ctypes.c_int
         lib.orc_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -93,15 +94,22 @@ def num_threads() -> int:
     return int(_load().orc_num_threads())
 
 
-def scan(x, g) -> np.ndarray:
-    """h_t = g_t h_{t-1} + (1 - g_t) x_t along axis 1 of [B, T, ...] arrays."""
+def scan(x, g, L: int = 0) -> np.ndarray:
+    """h_t = g_t h_{t-1} + (1 - g_t) x_t along axis 1 of [B, T, ...] arrays.
+
+    L > 0: chunk-local recurrence, the state restarts at every t with
+    t mod L == 0 (the original RAT's blocks); L == 0: the full sequence.
+    """
     x = _f64(x)
     g = _f64(g)
-    assert x.shape == g.shape and x.ndim >= 2
+    assert x.shape == g.shape and x.ndim >= 2 and L >= 0
     B, T = x.shape[0], x.shape[1]
     C = int(np.prod(x.shape[2:])) if x.ndim > 2 else 1
     h = np.empty_like(x)
-    _load().orc_scan(_p(x), _p(g), _p(h), B, T, C)
+    if L == 0:
+        _load().orc_scan(_p(x), _p(g), _p(h), B, T, C)
+    else:
+        _load().orc_scan_reset(_p(x), _p(g), _p(h), B, T, C, L)
     return h
 
 
@@ -158,8 +166,11 @@ def ring_row(b, h, p, H, W) -> int:
 class Cache:
     """fp64 mirror of the D-compressed cache plus the fp64 recurrent state."""
 
-    def __init__(self, B, H, Dh, T_max, D, W, dense_mask=None):
+    def __init__(self, B, H, Dh, T_max, D, W, dense_mask=None, L=0):
+        """L > 0: chunk-local recurrence (state zeroed at every t mod L == 0)."""
+        assert L >= 0
         self.B, self.H, self.Dh, self.T_max, self.D, self.W = B, H, Dh, T_max, D, W
+        self.L = L
         self.mask, self._mp = _mask(dense_mask, H)
         rows = cache_rows_total(B, H, T_max, D, dense_mask)
         self.Kc = np.zeros((rows, Dh))
@@ -186,7 +197,7 @@ class Cache:
         rc = _load().orc_decode_step(_p(q), _p(xk), _p(xv), _p(g), _p(self.state),
                                      _p(self.Kc), _p(self.Vc), _p(self.Kw), _p(self.Vw),
                                      _p(self.len, _L), _p(o), self.B, self.H, self.Dh,
-                                     self.T_max, self.D, self.W, self._mp)
+                                     self.T_max, self.D, self.W, self._mp, self.L)
         if rc != 0:
             raise RuntimeError("oracle decode: cache capacity exceeded")
         return o

@@ -27,7 +27,12 @@
  *     with the dilated set (each key once); W == 0 means no window;
  *   - scores q_t . hk_j / sqrt(Dh), softmax over the key set, output
  *     sum_j p_j hv_j; queries are not recurrent, keys/values are;
- *   - a dense head (dense_mask[h] != 0) uses D = 1.
+ *   - a dense head (dense_mask[h] != 0) uses D = 1;
+ *   - chunk-local variant (the original RAT that [zc] section 2.1 contrasts
+ *     with RAT+: each token recurs only inside its own block of L tokens):
+ *     the state is zeroed before position t whenever t mod L == 0, at
+ *     prefill and at decode alike; the key and value streams restart
+ *     together.
  *
  * Parity pins for every function live in the CPU test-suite (closed forms,
  * brute-force masks, dense causal attention from a library routine,
@@ -57,6 +62,28 @@ void orc_scan(const double* x, const double* g, double* h,
             double state = 0.0;                      /* h_{-1} = 0 */
             for (long t = 0; t < T; ++t) {
                 long i = (b * T + t) * C + c;
+                state = g[i] * state + (1.0 - g[i]) * x[i];
+                h[i] = state;
+            }
+        }
+    }
+}
+
+/* Chunk-local recurrence of the original RAT ([zc] section 2.1: the state
+ * restarts at every chunk of L tokens, L = D there): the same recurrence with
+ * h_{t-1} taken as 0 whenever t mod L == 0.  L <= 0 means no restart (the
+ * full-sequence recurrence of orc_scan). */
+void orc_scan_reset(const double* x, const double* g, double* h,
+                    long B, long T, long C, long L)
+{
+    long b;
+#pragma omp parallel for schedule(static)
+    for (b = 0; b < B; ++b) {
+        for (long c = 0; c < C; ++c) {
+            double state = 0.0;
+            for (long t = 0; t < T; ++t) {
+                long i = (b * T + t) * C + c;
+                if (L > 0 && t % L == 0) state = 0.0;    /* a chunk starts at t */
                 state = g[i] * state + (1.0 - g[i]) * x[i];
                 h[i] = state;
             }
@@ -295,7 +322,7 @@ int orc_decode_step(const double* q, const double* xk, const double* xv,
                     const double* g, double* state, double* Kc, double* Vc,
                     double* Kw, double* Vw, long* len, double* o,
                     long B, long H, long Dh, long T_max, long D, long W,
-                    const unsigned char* dense_mask)
+                    const unsigned char* dense_mask, long L)
 {
     const double scale = 1.0 / sqrt((double)Dh);
     int status = 0;
@@ -312,6 +339,9 @@ int orc_decode_step(const double* q, const double* xk, const double* xv,
             long i0 = (b * H + h) * Dh;
             double* sk = state + i0;
             double* sv = state + B * H * Dh + i0;
+            if (L > 0 && t % L == 0) {                /* chunk-local recurrence restarts */
+                for (long c = 0; c < Dh; ++c) { sk[c] = 0.0; sv[c] = 0.0; }
+            }
             orc_scan_step(xk + i0, g + i0, sk, Dh);
             orc_scan_step(xv + i0, g + i0, sv, Dh);
             long nk = 0;

@@ -2,6 +2,9 @@
 
 * recurrence: hand-worked fixture, g = 0 identity, constant-gate closed form
   (geometric sum), and the associative affine-map composition;
+* chunk-local recurrence: L = 1 closed form, the constant-gate closed form
+  restarted per block, L >= T equal to the full recurrence, blocks equal to
+  independent recurrences, and insensitivity to earlier blocks' inputs;
 * key sets: hand-worked fixture, an independent membership predicate, and a
   closed-form count;
 * attention: hand-worked fixture, dense causal attention from
@@ -70,6 +73,46 @@ def test_scan_associative_composition():
         end = A * carry + Bv
         np.testing.assert_allclose(h[:, hi - 1], end, rtol=1e-12, atol=1e-12)
         carry = end
+
+
+# ---------------------------------------------------- chunk-local recurrence
+def test_scan_reset_every_token_is_input_weighting():
+    x = RNG.standard_normal((2, 23, 7))
+    g = RNG.uniform(0, 1, x.shape)
+    h = oracle.scan(x, g, L=1)
+    np.testing.assert_allclose(h, (1 - g) * x, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("L", [3, 16, 64])
+def test_scan_reset_constant_gate_unit_input(L):
+    c, T = 0.8, 150
+    h = oracle.scan(np.ones((1, T, 1)), np.full((1, T, 1), c), L=L).ravel()
+    np.testing.assert_allclose(h, 1 - c ** (np.arange(T) % L + 1), rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("L", [41, 97, 1000])
+def test_scan_reset_longer_than_sequence_is_full(L):
+    x = RNG.standard_normal((2, 41, 5))
+    g = RNG.uniform(0, 1, x.shape)
+    assert np.array_equal(oracle.scan(x, g, L=L), oracle.scan(x, g))
+
+
+@pytest.mark.parametrize("L", [2, 7, 16])
+def test_scan_reset_blocks_are_independent(L):
+    B, T, C = 2, 53, 4
+    x = RNG.standard_normal((B, T, C))
+    g = RNG.uniform(0, 1, (B, T, C))
+    h = oracle.scan(x, g, L=L)
+    for lo in range(0, T, L):
+        hi = min(lo + L, T)
+        np.testing.assert_allclose(h[:, lo:hi], oracle.scan(x[:, lo:hi], g[:, lo:hi]),
+                                   rtol=0, atol=1e-15)
+    # inputs of earlier blocks never reach a later block
+    x2 = x.copy()
+    x2[:, : 2 * L] += 10.0
+    h2 = oracle.scan(x2, g, L=L)
+    assert np.array_equal(h2[:, 2 * L:], h[:, 2 * L:])
+    assert not np.array_equal(h2[:, :L], h[:, :L])
 
 
 # ---------------------------------------------------------------- key sets
@@ -229,6 +272,28 @@ def test_decode_continues_prefill(D, W, mask):
                 row = oracle.cache_row(b, h, s, H, N, D, mask)
                 np.testing.assert_allclose(cache.Kc[row], hk[b, s * Dd + Dd - 1, h], rtol=1e-12)
                 np.testing.assert_allclose(cache.Vc[row], hv[b, s * Dd + Dd - 1, h], rtol=1e-12)
+
+
+@pytest.mark.parametrize("L,T", [(4, 12), (5, 13), (1, 7), (16, 10)])
+def test_decode_chunk_local_continues_prefill(L, T):
+    """With chunk-local recurrence the decode step restarts the state at the
+    same positions as the prefill scan (blocks cross the prefill boundary)."""
+    B, n, H, Dh, D, W = 2, 11, 2, 8, 3, 2
+    N = T + n
+    q = RNG.standard_normal((B, N, H, Dh))
+    xk = RNG.standard_normal((B, N, H, Dh))
+    xv = RNG.standard_normal((B, N, H, Dh))
+    g = RNG.uniform(0, 1, (B, N, H, Dh))
+    hk, hv = oracle.scan(xk, g, L=L), oracle.scan(xv, g, L=L)
+    ref = oracle.attention(q, hk, hv, D, W)
+    cache = oracle.Cache(B, H, Dh, N, D, W, L=L)
+    cache.pack(hk[:, :T], hv[:, :T], state=np.stack([hk[:, T - 1], hv[:, T - 1]]))
+    for i in range(n):
+        t = T + i
+        o = cache.decode_step(q[:, t], xk[:, t], xv[:, t], g[:, t])
+        np.testing.assert_allclose(o, ref[:, t], rtol=1e-11, atol=1e-11)
+    np.testing.assert_allclose(cache.state, np.stack([hk[:, N - 1], hv[:, N - 1]]),
+                               rtol=1e-12, atol=1e-12)
 
 
 def test_decode_capacity_error():
