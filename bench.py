@@ -362,6 +362,41 @@ def measure_config(name, dev, steps, warmup, peaks):
     return out
 
 
+def measure_chunk_local(name, L_list, dev, steps, warmup, peaks):
+    """The key/value scan of one workload with the chunk-local recurrence (the
+    original RAT's blocks of L tokens) beside the full-sequence scan, timed
+    with CUDA events on the launching stream.  Reported beside the headline
+    line, not part of it."""
+    import recurrence_augmented_dilated_chunked_b200 as ratp
+    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
+    w = WORKLOADS[name]
+    stream = torch.cuda.current_stream(dev)
+    _, xk, xv, g = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.H, w.Dh, w.dtype,
+                                                        w.gate_mean, w.gate_std, seed=0))
+    hk, hv = torch.empty_like(xk), torch.empty_like(xv)
+    fs = torch.empty(2, w.B, w.H, w.Dh, dtype=torch.float32, device=dev)
+    ws = ratp.scan_workspace(w.B, w.T, w.H, w.Dh, xk.dtype, dev)
+    pc = prefill_counts(w)
+    out = {"workload": name}
+    for L in [0] + list(L_list):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for i in range(warmup + steps):
+            ev = evs[i - warmup] if i >= warmup else None
+            if ev:
+                ev[0].record(stream)
+            ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, final_state=fs, workspace=ws, L=L)
+            if ev:
+                ev[1].record(stream)
+        torch.cuda.synchronize()
+        ratp.last_error(dev)
+        ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+        gbs = pc["scan_bytes"] / (ms / 1e3) / 1e9
+        out["full_sequence" if L == 0 else "L%d" % L] = {"scan_ms": ms, "achieved_gbs": gbs,
+                                                         "frac_hbm": gbs / peaks["hbm_gbs"]}
+    del xk, xv, g, hk, hv, ws
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import recurrence_augmented_dilated_chunked_b200 as ratp
     from recurrence_augmented_dilated_chunked_b200 import (WORKLOADS, decode_context,
@@ -593,6 +628,8 @@ def run_ours(args, rank, world, local_rank):
         # the other workloads, measured after the timed region (not part of it)
         line["other_configs"] = {n: measure_config(n, dev, min(args.steps, 5), args.warmup, peaks)
                                  for n in OTHER_CONFIGS}
+        line["chunk_local_scan"] = measure_chunk_local(PREFILL, [wp.D, 1000], dev,
+                                                       min(args.steps, 5), args.warmup, peaks)
     if not args.no_cpu_baseline and world >= 1:
         line["cpu_baseline"] = oracle_sample()
     print(json.dumps(line), flush=True)

@@ -120,6 +120,28 @@ int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Chunk-local recurrence (the original RAT, which section 2.1 of the
+ * zhichai.net write-up "RAT+ 深度拆解" describes as the method RAT+ replaces:
+ * the sequence is cut into blocks of L tokens and each token recurs only
+ * inside its own block; there L = D).
+ *
+ * h_t = g_t * h_{t-1} + (1 - g_t) * x_t, with h_{t-1} taken as 0 whenever
+ * t mod L == 0; positions count from 0 at the first token of x.
+ * Arguments, layouts, workspace and errors are those of ratp_scan_prefill /
+ * ratp_scan_prefill_kv, plus L: L >= 1 is the block length; L == 0 (or any
+ * L >= T) gives the full-sequence recurrence; L < 0 is RATP_ERR_ARG.
+ * final_state receives h_{T-1}; a decode that continues from it must use a
+ * cache with the same L (ratp_cache_set_chunk_local).
+ * ---------------------------------------------------------------------- */
+int ratp_scan_prefill_chunk_local(const void* x, const void* g, void* h, float* final_state,
+                                  int B, int T, int H, int Dh, int dtype, int L,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+int ratp_scan_prefill_kv_chunk_local(const void* xk, const void* xv, const void* g,
+                                     void* hk, void* hv, float* final_state,
+                                     int B, int T, int H, int Dh, int dtype, int L,
+                                     void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * Allocation-free variant of ratp_scan_prefill_kv.  The paper has no
  * counterpart: this is a convenience of the library.
  *
@@ -203,6 +225,8 @@ typedef struct ratp_cache {
   int32_t B, H, Dh, T_max, D, W;
   int32_t split_keys;   /* keys per decode split */
   int32_t max_splits;   /* most decode splits any head can need (partial rows per (b, h)) */
+  int32_t reset_L;      /* chunk-local recurrence block (0 = full sequence); set by
+                           ratp_cache_set_chunk_local */
   uint8_t dense[RATP_MAX_HEADS];
 } ratp_cache;
 
@@ -223,8 +247,16 @@ int ratp_cache_init(ratp_cache* c, void* buffer, size_t bytes,
  * final_state (ratp_scan_prefill_kv writes the [2][B][H][Dh] decode layout). */
 int ratp_cache_pack(ratp_cache* c, const void* hk, const void* hv, int T, void* stream);
 
+/* Selects the recurrence that ratp_decode_step continues: L == 0 (the
+ * default that ratp_cache_init sets) is the full-sequence recurrence; L >= 1
+ * is the chunk-local recurrence of ratp_scan_prefill_kv_chunk_local, whose
+ * state restarts at every position t with t mod L == 0.  Host-only: writes
+ * c->reset_L and launches nothing.  Errors: ARG (null c, L < 0). */
+int ratp_cache_set_chunk_local(ratp_cache* c, int L);
+
 /* One decode token for every sequence (fused): state <- g*state + (1-g)*x for
- * the key and value streams (fp32 state [2][B][H][Dh], in/out); the new
+ * the key and value streams (fp32 state [2][B][H][Dh], in/out; the state is
+ * first zeroed where t mod c->reset_L == 0 for a chunk-local cache); the new
  * recurrent key/value is appended to Kc/Vc when t mod D_h == D_h - 1 and
  * always written to the ring; o = attention of q over the cached dilated
  * slots s < t / D_h, the window positions t-W < p < t not among them, and the

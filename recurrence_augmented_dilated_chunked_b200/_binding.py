@@ -39,6 +39,7 @@ class CacheStruct(ctypes.Structure):
         ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("Dh", ctypes.c_int32),
         ("T_max", ctypes.c_int32), ("D", ctypes.c_int32), ("W", ctypes.c_int32),
         ("split_keys", ctypes.c_int32), ("max_splits", ctypes.c_int32),
+        ("reset_L", ctypes.c_int32),
         ("dense", ctypes.c_uint8 * MAX_HEADS),
     ]
 
@@ -55,12 +56,15 @@ _SIGS = {
     "ratp_scan_workspace_bytes": ([_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "ratp_scan_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "ratp_scan_prefill_kv": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
+    "ratp_scan_prefill_chunk_local": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
+    "ratp_scan_prefill_kv_chunk_local": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "ratp_scan_prefill_kv_noalloc": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P], _I),
     "ratp_dilated_attn_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_simt": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_cache_bytes": ([_I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)], _I),
     "ratp_cache_init": ([ctypes.POINTER(CacheStruct), _P, _SZ, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ratp_cache_pack": ([ctypes.POINTER(CacheStruct), _P, _P, _I, _P], _I),
+    "ratp_cache_set_chunk_local": ([ctypes.POINTER(CacheStruct), _I], _I),
     "ratp_decode_step": ([_P, _P, _P, _P, _P, ctypes.POINTER(CacheStruct), _P, _I, _I, _P, _P], _I),
 }
 
@@ -136,8 +140,10 @@ def scan_workspace(B, T, H, Dh, dtype, device) -> torch.Tensor:
     return ws
 
 
-def scan_prefill(x, g, out=None, final_state=None, workspace=None):
-    """h = forget-gate scan of x with gates g over axis 1 of [B, T, H, Dh]."""
+def scan_prefill(x, g, out=None, final_state=None, workspace=None, L=0):
+    """h = forget-gate scan of x with gates g over axis 1 of [B, T, H, Dh].
+
+    L >= 1: chunk-local recurrence (the state restarts at t mod L == 0)."""
     lib = load_library()
     _need(x, "x")
     _need(g, "g", x.dtype)
@@ -148,14 +154,21 @@ def scan_prefill(x, g, out=None, final_state=None, workspace=None):
     if final_state is not None:
         _need(final_state, "final_state", torch.float32)
     ws = workspace if workspace is not None else scan_workspace(B, T, H, Dh, x.dtype, x.device)
-    _check("ratp_scan_prefill", lib.ratp_scan_prefill(
-        _ptr(x), _ptr(g), _ptr(out), _ptr(final_state), B, T, H, Dh, _DTYPE[x.dtype],
-        _ptr(ws), ws.numel(), _stream(x)))
+    if L:
+        _check("ratp_scan_prefill_chunk_local", lib.ratp_scan_prefill_chunk_local(
+            _ptr(x), _ptr(g), _ptr(out), _ptr(final_state), B, T, H, Dh, _DTYPE[x.dtype], int(L),
+            _ptr(ws), ws.numel(), _stream(x)))
+    else:
+        _check("ratp_scan_prefill", lib.ratp_scan_prefill(
+            _ptr(x), _ptr(g), _ptr(out), _ptr(final_state), B, T, H, Dh, _DTYPE[x.dtype],
+            _ptr(ws), ws.numel(), _stream(x)))
     return out
 
 
-def scan_prefill_kv(xk, xv, g, hk=None, hv=None, final_state=None, workspace=None):
-    """(hk, hv) = scans of xk and xv sharing the gate tensor g (one pass)."""
+def scan_prefill_kv(xk, xv, g, hk=None, hv=None, final_state=None, workspace=None, L=0):
+    """(hk, hv) = scans of xk and xv sharing the gate tensor g (one pass).
+
+    L >= 1: chunk-local recurrence (the state restarts at t mod L == 0)."""
     lib = load_library()
     _need(xk, "xk")
     _need(xv, "xv", xk.dtype)
@@ -168,9 +181,14 @@ def scan_prefill_kv(xk, xv, g, hk=None, hv=None, final_state=None, workspace=Non
     if final_state is not None:
         _need(final_state, "final_state", torch.float32)
     ws = workspace if workspace is not None else scan_workspace(B, T, H, Dh, xk.dtype, xk.device)
-    _check("ratp_scan_prefill_kv", lib.ratp_scan_prefill_kv(
-        _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(final_state),
-        B, T, H, Dh, _DTYPE[xk.dtype], _ptr(ws), ws.numel(), _stream(xk)))
+    if L:
+        _check("ratp_scan_prefill_kv_chunk_local", lib.ratp_scan_prefill_kv_chunk_local(
+            _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(final_state),
+            B, T, H, Dh, _DTYPE[xk.dtype], int(L), _ptr(ws), ws.numel(), _stream(xk)))
+    else:
+        _check("ratp_scan_prefill_kv", lib.ratp_scan_prefill_kv(
+            _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(final_state),
+            B, T, H, Dh, _DTYPE[xk.dtype], _ptr(ws), ws.numel(), _stream(xk)))
     return hk, hv
 
 
@@ -244,7 +262,8 @@ def sm_count() -> int:
 class KVCache:
     """D-compressed KV cache for decode (one device buffer, see ``ratp.h``)."""
 
-    def __init__(self, B, H, Dh, T_max, D, W=0, head_mask=None, device="cuda"):
+    def __init__(self, B, H, Dh, T_max, D, W=0, head_mask=None, device="cuda", L=0):
+        """L >= 1: decode continues a chunk-local recurrence of block L."""
         lib = load_library()
         self.B, self.H, self.Dh, self.T_max, self.D, self.W = B, H, Dh, T_max, D, W
         self.head_mask = [1 if v else 0 for v in head_mask] if head_mask is not None else None
@@ -256,6 +275,8 @@ class KVCache:
         _check("ratp_cache_init", lib.ratp_cache_init(
             ctypes.byref(self.c), _ptr(self.buffer), n.value, B, H, Dh, T_max, D, W, mp,
             _stream(self.buffer)))
+        self.L = int(L)
+        _check("ratp_cache_set_chunk_local", lib.ratp_cache_set_chunk_local(ctypes.byref(self.c), self.L))
 
     def _view(self, addr, numel, dtype):
         off = addr - self.buffer.data_ptr()

@@ -11,7 +11,8 @@
 //   [i*split_keys, (i+1)*split_keys) with 16-byte loads, a half-warp per key
 //   (Dh = 128) and an fp32 online softmax per half-warp.
 //   Split 0 additionally performs the recurrence step for the k and v streams
-//   (fp32 state, in place), appends the bf16-rounded new key/value to Kc/Vc
+//   (fp32 state, in place; with a chunk-local recurrence of block reset_L the
+//   state is taken as zero at t mod reset_L == 0), appends the bf16-rounded new key/value to Kc/Vc
 //   when t mod D_h = D_h-1, writes it into ring row t mod W, and attends to it
 //   (the query's own key).  None of these rows is read by any CTA of the
 //   same step, so there is no intra-step race.
@@ -42,6 +43,7 @@ struct Params {
   uint32_t* counters;           // [B*H] per (b, h), then [B] per batch item
   long long rows_per_b;
   int B, H, D, W, T_max, split_keys, max_splits;
+  int reset_L;                  // chunk-local recurrence: state restarts at t mod reset_L == 0; 0 = never
   float scale_log2;
   int splits_per_b;             // CTAs per batch item: sum over heads of split_base
   int split_base[RATP_MAX_HEADS + 1];   // first CTA (within a batch item) of each head
@@ -128,7 +130,8 @@ decode_kernel(const Params p) {
         float* st = p.state + ((long long)s * p.B * p.H + bh) * DH + ch;
         const float x = __bfloat162float((s == 0 ? p.xk : p.xv)[bh * DH + ch]);
         const float gg = __bfloat162float(p.g[bh * DH + ch]);
-        const float hn = fmaf(gg, *st - x, x);
+        const float prev = (p.reset_L > 0 && t % p.reset_L == 0) ? 0.f : *st;
+        const float hn = fmaf(gg, prev - x, x);
         *st = hn;
         const __nv_bfloat16 hb = __float2bfloat16_rn(hn);
         (s == 0 ? s_self_k : s_self_v)[ch] = __bfloat162float(hb);

@@ -109,9 +109,9 @@ unsigned int next_scan_epoch() {
   return e;
 }
 
-template <typename T, int NS>
+template <typename T, int NS, bool RESET>
 int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
-                int B, int Tn, int H, int Dh, const ScanGeom& geo,
+                int B, int Tn, int H, int Dh, int reset_L, const ScanGeom& geo,
                 void* ws, size_t ws_bytes, cudaStream_t st) {
   if (geo.n_chunks == 0) return RATP_OK;
   if (ws == nullptr || !aligned16(ws)) return ws == nullptr ? RATP_ERR_ARG : RATP_ERR_ALIGN;
@@ -122,6 +122,7 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   p.ws = scan::carve(ws, geo.n_chunks, NS);
   p.epoch = next_scan_epoch();
   p.B = B; p.Tn = Tn; p.C = H * Dh;
+  p.reset_L = reset_L;
   p.slabs = geo.slabs; p.n_chains = geo.n_chains; p.n_chunks_t = geo.n_chunks_t;
   const int C = H * Dh, rows = scan::Shape<T>::kChunk;
   CUtensorMap tg, tx0, tx1;
@@ -133,16 +134,28 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
     tx1 = tx0;
   }
   constexpr int smem = scan::Smem<T, NS>::kBytes;
-  if (!ensure_smem(scan::scan_kernel<T, NS>, smem)) return RATP_ERR_CUDA;
+  auto kernel = scan::scan_kernel<T, NS, scan::kRows, RESET>;
+  if (!ensure_smem(kernel, smem)) return RATP_ERR_CUDA;
   cudaError_t e = cudaMemsetAsync(ws, 0, scan::reset_bytes(geo.n_chunks), st);
   if (e != cudaSuccess) return RATP_ERR_CUDA;
   // one CTA per chunk; chunk tickets, not block indices, fix the order
-  scan::scan_kernel<T, NS><<<(unsigned)geo.n_chunks, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);
+  kernel<<<(unsigned)geo.n_chunks, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);
   return launch_status();
 }
 
+template <typename E, bool RESET>
+int launch_scan_ns(int NS, const void* const* x, const void* g, void* const* h, float* fs,
+                   int B, int T, int H, int Dh, int reset_L, const ScanGeom& geo,
+                   void* ws, size_t ws_bytes, cudaStream_t st) {
+  return NS == 1 ? launch_scan<E, 1, RESET>(x, g, h, fs, B, T, H, Dh, reset_L, geo, ws, ws_bytes, st)
+                 : launch_scan<E, 2, RESET>(x, g, h, fs, B, T, H, Dh, reset_L, geo, ws, ws_bytes, st);
+}
+
+// reset_L: 0 = the full-sequence recurrence, >= 1 = chunk-local blocks of reset_L tokens
 int scan_common(int NS, const void* const* x, const void* g, void* const* h, float* fs,
-                int B, int T, int H, int Dh, int dtype, void* ws, size_t ws_bytes, void* stream) {
+                int B, int T, int H, int Dh, int dtype, int reset_L,
+                void* ws, size_t ws_bytes, void* stream) {
+  if (reset_L < 0) return RATP_ERR_ARG;
   ScanGeom geo;
   int rc = scan_geom(B, T, H, Dh, dtype, &geo);
   if (rc) return rc;
@@ -155,12 +168,14 @@ int scan_common(int NS, const void* const* x, const void* g, void* const* h, flo
   if (!aligned16(g)) return RATP_ERR_ALIGN;
   if (fs != nullptr && !aligned16(fs)) return RATP_ERR_ALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // a block at least as long as the sequence never restarts after t = 0
+  const bool reset = reset_L > 0 && reset_L < T;
   if (dtype == RATP_BF16) {
-    return NS == 1 ? launch_scan<__nv_bfloat16, 1>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st)
-                   : launch_scan<__nv_bfloat16, 2>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st);
+    return reset ? launch_scan_ns<__nv_bfloat16, true>(NS, x, g, h, fs, B, T, H, Dh, reset_L, geo, ws, ws_bytes, st)
+                 : launch_scan_ns<__nv_bfloat16, false>(NS, x, g, h, fs, B, T, H, Dh, 0, geo, ws, ws_bytes, st);
   }
-  return NS == 1 ? launch_scan<float, 1>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st)
-                 : launch_scan<float, 2>(x, g, h, fs, B, T, H, Dh, geo, ws, ws_bytes, st);
+  return reset ? launch_scan_ns<float, true>(NS, x, g, h, fs, B, T, H, Dh, reset_L, geo, ws, ws_bytes, st)
+               : launch_scan_ns<float, false>(NS, x, g, h, fs, B, T, H, Dh, 0, geo, ws, ws_bytes, st);
 }
 
 // ---- head masks -------------------------------------------------------------
@@ -448,7 +463,15 @@ int ratp_scan_prefill(const void* x, const void* g, void* h, float* final_state,
                       void* workspace, size_t workspace_bytes, void* stream) {
   const void* xs[1] = {x};
   void* hs[1] = {h};
-  return scan_common(1, xs, g, hs, final_state, B, T, H, Dh, dtype, workspace, workspace_bytes, stream);
+  return scan_common(1, xs, g, hs, final_state, B, T, H, Dh, dtype, 0, workspace, workspace_bytes, stream);
+}
+
+int ratp_scan_prefill_chunk_local(const void* x, const void* g, void* h, float* final_state,
+                                  int B, int T, int H, int Dh, int dtype, int L,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  const void* xs[1] = {x};
+  void* hs[1] = {h};
+  return scan_common(1, xs, g, hs, final_state, B, T, H, Dh, dtype, L, workspace, workspace_bytes, stream);
 }
 
 int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
@@ -457,7 +480,16 @@ int ratp_scan_prefill_kv(const void* xk, const void* xv, const void* g,
                          void* workspace, size_t workspace_bytes, void* stream) {
   const void* xs[2] = {xk, xv};
   void* hs[2] = {hk, hv};
-  return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, workspace, workspace_bytes, stream);
+  return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, 0, workspace, workspace_bytes, stream);
+}
+
+int ratp_scan_prefill_kv_chunk_local(const void* xk, const void* xv, const void* g,
+                                     void* hk, void* hv, float* final_state,
+                                     int B, int T, int H, int Dh, int dtype, int L,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+  const void* xs[2] = {xk, xv};
+  void* hs[2] = {hk, hv};
+  return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, L, workspace, workspace_bytes, stream);
 }
 
 int ratp_scan_prefill_kv_noalloc(const void* xk, const void* xv, const void* g,
@@ -473,7 +505,7 @@ int ratp_scan_prefill_kv_noalloc(const void* xk, const void* xv, const void* g,
   if (rc) return rc;
   const void* xs[2] = {xk, xv};
   void* hs[2] = {hk, hv};
-  return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, ws,
+  return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, 0, ws,
                      (size_t)RATP_NOALLOC_SCRATCH_BYTES, stream);
 }
 
@@ -530,6 +562,7 @@ int ratp_cache_init(ratp_cache* c, void* buffer, size_t bytes, int B, int H, int
   c->B = B; c->H = H; c->Dh = Dh; c->T_max = T_max; c->D = D; c->W = W;
   c->split_keys = L.split_keys;
   c->max_splits = L.max_splits;
+  c->reset_L = 0;
   for (int h = 0; h < H; ++h) c->dense[h] = (head_mask != nullptr && head_mask[h] != 0) ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(c->len, 0, (size_t)B * 4, st) != cudaSuccess) return RATP_ERR_CUDA;
@@ -568,10 +601,17 @@ int ratp_cache_pack(ratp_cache* c, const void* hk, const void* hv, int T, void* 
   return launch_status();
 }
 
+int ratp_cache_set_chunk_local(ratp_cache* c, int L) {
+  if (!c || L < 0) return RATP_ERR_ARG;
+  c->reset_L = L;
+  return RATP_OK;
+}
+
 int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* g,
                      float* state, ratp_cache* c, void* o,
                      int D, int W, const uint8_t* head_mask, void* stream) {
   if (!q || !xk || !xv || !g || !state || !c || !o) return RATP_ERR_ARG;
+  if (c->reset_L < 0) return RATP_ERR_ARG;
   if (!aligned16(q) || !aligned16(xk) || !aligned16(xv) || !aligned16(g) || !aligned16(state) ||
       !aligned16(o))
     return RATP_ERR_ALIGN;
@@ -594,6 +634,7 @@ int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* 
   p.B = c->B; p.H = c->H; p.D = c->D; p.W = c->W; p.T_max = c->T_max;
   p.split_keys = c->split_keys;
   p.max_splits = c->max_splits;
+  p.reset_L = c->reset_L;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)c->Dh);
   int rc = read_mask(c->dense, c->H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
   if (rc) return rc;

@@ -25,6 +25,15 @@
 //   * every wait is bounded (spin_timeout()); on expiry the kernel records
 //     RATP_ERR_TIMEOUT, sets a kernel-wide abort word so that no other CTA
 //     keeps waiting, and finishes with a zero carry.
+//
+// Chunk-local variant (RESET; the original RAT that section 2.1 of the same
+// write-up contrasts with RAT+, where a token recurs only inside its block of
+// reset_L tokens): the step of a token t with t mod reset_L == 0 becomes the
+// map (0, (1 - g) x).  Only those steps change; the composition, the in-chunk
+// scan and the look-back are the same maps.  A chunk whose first token
+// restarts needs no carry and skips the look-back; otherwise the look-back
+// stops at the predecessor holding the last restart (its aggregate slope is
+// exactly 0), so no chain waits further back than one block.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -115,6 +124,7 @@ struct Params {
   Workspace ws;
   unsigned int epoch;     // nonzero, unique per launch
   int B, Tn, C;           // Tn tokens, C = H * Dh channels per token
+  int reset_L;            // chunk-local block length (RESET kernels only, >= 1)
   int slabs;              // C / 64
   int n_chains;           // B * slabs
   int n_chunks_t;         // chunks along T
@@ -130,7 +140,7 @@ struct Smem {
   static constexpr int kBytes = kData + kScan + 128;                       // + alignment
 };
 
-template <typename T, int NS, int R = kRows>
+template <typename T, int NS, int R = kRows, bool RESET = false>
 __global__ void __launch_bounds__(kThreads, 2)
 scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x0,
             const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ Params<T, NS> p) {
@@ -186,6 +196,11 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   const long long row_stride = p.C;
   const long long base = ((long long)b * p.Tn) * row_stride + (long long)slab * kSlab + lane_c * V;
   const int soff = grp * R * kSlab + lane_c * V;   // element offset of row 0 in a tile
+  // rows r of this thread whose token restarts the recurrence (bit r)
+  unsigned int rmask = 0u;
+  if (RESET) {
+    for (int r = (p.reset_L - t0 % p.reset_L) % p.reset_L; r < R; r += p.reset_L) rmask |= 1u << r;
+  }
 
   {
     // one thread waits for the tiles (bounded; the clock and the abort word
@@ -229,6 +244,14 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     if (r < nrows) {
+      if (RESET && ((rmask >> r) & 1u)) {    // restart: forget the rows before
+#pragma unroll
+        for (int i = 0; i < V2; ++i) {
+          la[i] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int s = 0; s < NS; ++s) lb[s][i] = make_float2(0.f, 0.f);
+        }
+      }
       float2 gf[V2];
       Elem<T>::unpack2(*reinterpret_cast<const uint4*>(s_g + soff + r * kSlab), gf);
 #pragma unroll
@@ -370,7 +393,9 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
         put_word(dst + (3 + 2 * s) * kDescLanes, s_tot_b[s][c0 + 1], p.epoch);
       }
     }
-    if (chunk > 0) {
+    // a chunk whose first token restarts the recurrence needs no carry
+    const bool restart = RESET && ((long long)chunk * L) % p.reset_L == 0;
+    if (chunk > 0 && !restart) {
       // composite map of the predecessors composed so far: x -> ca x + cb
       float ca0 = 1.f, ca1 = 1.f;
       int top = chunk - 1;                      // nearest predecessor not yet composed
@@ -440,6 +465,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
           }
           break;
         }
+        if (RESET && ca0 == 0.f && ca1 == 0.f) break;   // composed the last restart
         top -= n;
       }
     }
@@ -472,6 +498,12 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   for (int r = 0; r < R; ++r) {
     if (r < nrows) {
       const int t = t0 + r;
+      if (RESET && ((rmask >> r) & 1u)) {
+#pragma unroll
+        for (int s = 0; s < NS; ++s)
+#pragma unroll
+          for (int i = 0; i < V2; ++i) hs[s][i] = make_float2(0.f, 0.f);
+      }
       float2 gf[V2];
       Elem<T>::unpack2(*reinterpret_cast<const uint4*>(s_g + soff + r * kSlab), gf);
 #pragma unroll

@@ -113,6 +113,22 @@ def test_scan_rejects_bad_arguments_on_host(lib):
     assert lib.ratp_scan_prefill(None, None, None, None, 1, 0, 1, 64, 1, None, 0, None) == 0
 
 
+def test_chunk_local_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)
+    # a negative block length is refused before anything else is looked at
+    assert lib.ratp_scan_prefill_kv_chunk_local(p, p, p, p, p, None, 1, 8, 1, 64, 1, -1,
+                                                p, 1 << 20, None) == 1
+    assert lib.ratp_scan_prefill_chunk_local(p, p, p, None, 1, 8, 1, 64, 1, -5, p, 1 << 20, None) == 1
+    assert lib.ratp_scan_prefill_chunk_local(None, p, p, None, 1, 8, 1, 64, 1, 4, p, 1 << 20, None) == 1
+    assert lib.ratp_scan_prefill_kv_chunk_local(None, None, None, None, None, None, 1, 0, 1, 64, 1, 4,
+                                                None, 0, None) == 0
+    c = _binding.CacheStruct()
+    assert lib.ratp_cache_set_chunk_local(ctypes.byref(c), -1) == 1
+    assert lib.ratp_cache_set_chunk_local(None, 4) == 1
+    assert lib.ratp_cache_set_chunk_local(ctypes.byref(c), 16) == 0 and c.reset_L == 16
+    assert lib.ratp_cache_set_chunk_local(ctypes.byref(c), 0) == 0 and c.reset_L == 0
+
+
 def test_decode_rejects_mismatched_cache_on_host(lib):
     c = _binding.CacheStruct()
     c.D, c.W, c.H = 4, 0, 2
