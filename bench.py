@@ -397,6 +397,79 @@ def measure_chunk_local(name, L_list, dev, steps, warmup, peaks):
     return out
 
 
+# A 1.5B-like stack of 24 sequence mixers for the layer-wise hybrid: dense
+# layers at 0 (input) and 12 (middle), every other layer at D = 64 with a
+# 128-token window; decode from 32K-token contexts, 16 sequences.
+STACK = {"name": "bf16_1p5b_stack24_decode_ctx32768", "layers": 24, "dense_layers": (0, 12),
+         "B": 16, "H": 16, "Dh": 128, "D": 64, "W": 128, "ctx": 32768, "steps": 16}
+
+
+def measure_layer_stack(dev, replays, warmup, peaks):
+    """Decode token steps through the whole layer stack, each token step one
+    ``ratp_decode_step_layers`` call, 16 token steps captured in one CUDA
+    graph.  Caches are filled on the device with N(0, 1) rows (the values do
+    not change the work).  Reported beside the headline line."""
+    import recurrence_augmented_dilated_chunked_b200 as ratp
+    from recurrence_augmented_dilated_chunked_b200 import Workload, decode_inputs
+    S = STACK
+    n, B, H, Dh, ctx = S["steps"], S["B"], S["H"], S["Dh"], S["ctx"]
+    gen = torch.Generator(dev).manual_seed(5)
+    dq, dxk, dxv, dg = (t.to(dev) for t in decode_inputs(n, B, H, Dh, "bf16", 2.0, 1.5, seed=6))
+    layers, kinds = [], []
+    for li in range(S["layers"]):
+        dense = li in S["dense_layers"]
+        D, W = (1, 0) if dense else (S["D"], S["W"])
+        cache = ratp.KVCache(B, H, Dh, ctx + n, D, W, device=dev)
+        for which in ("k", "v"):
+            rows = cache.dil_rows(which)
+            rows.copy_(torch.randn(rows.shape, generator=gen, device=dev, dtype=torch.float32))
+            if W:
+                ring = cache.ring(which)
+                ring.copy_(torch.randn(ring.shape, generator=gen, device=dev, dtype=torch.float32))
+        state0 = torch.randn(2, B, H, Dh, generator=gen, device=dev, dtype=torch.float32)
+        out = torch.empty(n, B, H, Dh, dtype=torch.bfloat16, device=dev)
+        layers.append((cache, state0, state0.clone(), out))
+        kinds.append(Workload("stack", "bf16", B=B, T=0, H=H, Dh=Dh, D=D, W=W, gate_mean=2.0,
+                              gate_std=1.5, decode_steps=n, decode_ctx=ctx))
+
+    def burst():
+        for cache, s0, st, _ in layers:
+            cache.lengths().fill_(ctx)
+            st.copy_(s0)
+        for i in range(n):
+            ratp.decode_step_layers([(c, dq[i], dxk[i], dxv[i], dg[i], st, o[i])
+                                     for c, _, st, o in layers])
+
+    burst()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        burst()
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(warmup):
+        graph.replay()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(replays)]
+    for e in evs:
+        e[0].record(stream)
+        graph.replay()
+        e[1].record(stream)
+    torch.cuda.synchronize()
+    ratp.last_error(dev)
+    # the resets at the start of a burst are part of the replay; they move
+    # 2 * 24 small state copies, negligible beside the cache reads
+    ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs) / n
+    alg = sum(decode_bytes_per_step(w, ctx + i) for w in kinds for i in range(n)) / n
+    gbs = alg / (ms / 1e3) / 1e9
+    cache_bytes = sum(c.buffer.numel() for c, _, _, _ in layers)
+    del graph, layers
+    return {"workload": S["name"], "layers": S["layers"], "dense_layers": list(S["dense_layers"]),
+            "B": B, "H": H, "Dh": Dh, "D": S["D"], "W": S["W"], "ctx": ctx,
+            "token_steps_per_graph": n, "launches_per_token_step": S["layers"],
+            "ms_per_token_step": ms, "tokens_per_s": B / (ms / 1e3),
+            "alg_bytes_per_token_step": alg, "achieved_gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+            "cache_bytes": cache_bytes}
+
+
 def run_ours(args, rank, world, local_rank):
     import recurrence_augmented_dilated_chunked_b200 as ratp
     from recurrence_augmented_dilated_chunked_b200 import (WORKLOADS, decode_context,
@@ -630,6 +703,7 @@ def run_ours(args, rank, world, local_rank):
                                  for n in OTHER_CONFIGS}
         line["chunk_local_scan"] = measure_chunk_local(PREFILL, [wp.D, 1000], dev,
                                                        min(args.steps, 5), args.warmup, peaks)
+        line["layer_stack_decode"] = measure_layer_stack(dev, min(args.steps, 5), args.warmup, peaks)
     if not args.no_cpu_baseline and world >= 1:
         line["cpu_baseline"] = oracle_sample()
     print(json.dumps(line), flush=True)

@@ -269,6 +269,36 @@ int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* 
                      float* state, ratp_cache* c, void* o,
                      int D, int W, const uint8_t* head_mask, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Decode token step of a stack of layers (layer-wise hybrid, write-up
+ * section 6: a few dense layers, e.g. the input layer 0 and the middle layer
+ * 12, among dilated ones).  Each layer has its own cache, so its own D, W,
+ * head mask and recurrence (ratp_cache_init, ratp_cache_set_chunk_local);
+ * layers may differ in all of them.
+ *
+ * For l = 0 .. n_layers-1 in order, performs ratp_decode_step on
+ * layers[l] with the D, W and head mask of layers[l].cache, all on `stream`
+ * (each launch may start while the previous layer's kernel drains and waits
+ * for its completion before touching memory).  The whole call is one token
+ * step and can be captured into one CUDA graph.  The array and the structs
+ * are read on the host during the call only; every pointer in them is a
+ * device pointer with the meaning, layout and ownership of ratp_decode_step.
+ * Errors: ARG (n_layers < 0, layers NULL with n_layers > 0, a NULL field),
+ * ALIGN, SHAPE; on the first failing layer the call returns its status and
+ * launches no later layer (earlier layers' launches stand).
+ * ---------------------------------------------------------------------- */
+typedef struct ratp_decode_layer {
+  const void* q;      /* bf16 [B][H][Dh] */
+  const void* xk;     /* bf16 [B][H][Dh] */
+  const void* xv;     /* bf16 [B][H][Dh] */
+  const void* g;      /* bf16 [B][H][Dh], gates in (0, 1) */
+  float* state;       /* fp32 [2][B][H][Dh], in/out */
+  ratp_cache* cache;  /* this layer's cache (host struct, device buffers) */
+  void* o;            /* bf16 [B][H][Dh], out */
+} ratp_decode_layer;
+
+int ratp_decode_step_layers(const ratp_decode_layer* layers, int n_layers, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -13,6 +13,7 @@ from ._binding import (  # noqa: F401
     dilated_attn_prefill,
     dilated_attn_prefill_simt,
     debug_fault,
+    decode_step_layers,
     exported_symbols,
     last_error,
     load_library,

@@ -44,6 +44,15 @@ class CacheStruct(ctypes.Structure):
     ]
 
 
+class DecodeLayerStruct(ctypes.Structure):
+    """Mirror of ``struct ratp_decode_layer``."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("xk", ctypes.c_void_p), ("xv", ctypes.c_void_p),
+        ("g", ctypes.c_void_p), ("state", ctypes.c_void_p),
+        ("cache", ctypes.POINTER(CacheStruct)), ("o", ctypes.c_void_p),
+    ]
+
+
 _lib = None
 _lock = threading.Lock()
 
@@ -66,6 +75,7 @@ _SIGS = {
     "ratp_cache_pack": ([ctypes.POINTER(CacheStruct), _P, _P, _I, _P], _I),
     "ratp_cache_set_chunk_local": ([ctypes.POINTER(CacheStruct), _I], _I),
     "ratp_decode_step": ([_P, _P, _P, _P, _P, ctypes.POINTER(CacheStruct), _P, _I, _I, _P, _P], _I),
+    "ratp_decode_step_layers": ([ctypes.POINTER(DecodeLayerStruct), _I, _P], _I),
 }
 
 
@@ -330,3 +340,23 @@ class KVCache:
             self.D, self.W, ctypes.cast(self._mask_buf, ctypes.c_void_p) if self._mask_buf is not None else None,
             _stream(q)))
         return out
+
+
+def decode_step_layers(layers):
+    """One decode token through a stack of layers in one call.
+
+    layers: sequence of (cache, q, xk, xv, g, state, out) with ``cache`` a
+    ``KVCache`` (its own D, W, head mask and recurrence), q/xk/xv/g/out bf16
+    [B, H, Dh] and state fp32 [2, B, H, Dh] (updated in place).  The layers
+    run in order on the current stream of the first q.
+    """
+    n = len(layers)
+    arr = (DecodeLayerStruct * max(n, 1))()
+    for i, (cache, q, xk, xv, g, state, out) in enumerate(layers):
+        for t, nm in ((q, "q"), (xk, "xk"), (xv, "xv"), (g, "g"), (out, "out")):
+            _need(t, nm, torch.bfloat16)
+        _need(state, "state", torch.float32)
+        arr[i] = DecodeLayerStruct(q.data_ptr(), xk.data_ptr(), xv.data_ptr(), g.data_ptr(),
+                                   state.data_ptr(), ctypes.pointer(cache.c), out.data_ptr())
+    stream = _stream(layers[0][1]) if n else None
+    _check("ratp_decode_step_layers", load_library().ratp_decode_step_layers(arr, n, stream))

@@ -607,15 +607,20 @@ int ratp_cache_set_chunk_local(ratp_cache* c, int L) {
   return RATP_OK;
 }
 
-int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* g,
-                     float* state, ratp_cache* c, void* o,
-                     int D, int W, const uint8_t* head_mask, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// One decode step of one layer: the checks and the launch behind
+// ratp_decode_step and ratp_decode_step_layers (the cache's own D, W and
+// head mask).
+int decode_launch(const void* q, const void* xk, const void* xv, const void* g,
+                  float* state, const ratp_cache* c, void* o, cudaStream_t st) {
   if (!q || !xk || !xv || !g || !state || !c || !o) return RATP_ERR_ARG;
   if (c->reset_L < 0) return RATP_ERR_ARG;
   if (!aligned16(q) || !aligned16(xk) || !aligned16(xv) || !aligned16(g) || !aligned16(state) ||
       !aligned16(o))
     return RATP_ERR_ALIGN;
-  if (!cache_matches(c, D, W, head_mask)) return RATP_ERR_ARG;
   decode::Params p;
   p.q = static_cast<const __nv_bfloat16*>(q);
   p.xk = static_cast<const __nv_bfloat16*>(xk);
@@ -638,7 +643,6 @@ int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* 
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)c->Dh);
   int rc = read_mask(c->dense, c->H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
   if (rc) return rc;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   // per-head split counts: the most keys head h can hold, over split_keys
   p.split_base[0] = 0;
   for (int h = 0; h < c->H; ++h) {
@@ -669,6 +673,29 @@ int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* 
                                  : cudaLaunchKernelEx(&cfg, decode::decode_kernel<64>, p);
   if (e != cudaSuccess) return RATP_ERR_CUDA;
   return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+int ratp_decode_step(const void* q, const void* xk, const void* xv, const void* g,
+                     float* state, ratp_cache* c, void* o,
+                     int D, int W, const uint8_t* head_mask, void* stream) {
+  if (!q || !xk || !xv || !g || !state || !c || !o) return RATP_ERR_ARG;
+  if (!cache_matches(c, D, W, head_mask)) return RATP_ERR_ARG;
+  return decode_launch(q, xk, xv, g, state, c, o, static_cast<cudaStream_t>(stream));
+}
+
+int ratp_decode_step_layers(const ratp_decode_layer* layers, int n_layers, void* stream) {
+  if (n_layers < 0 || (n_layers > 0 && layers == nullptr)) return RATP_ERR_ARG;
+  for (int l = 0; l < n_layers; ++l) {
+    const ratp_decode_layer& L = layers[l];
+    const int rc = decode_launch(L.q, L.xk, L.xv, L.g, L.state, L.cache, L.o,
+                                 static_cast<cudaStream_t>(stream));
+    if (rc) return rc;
+  }
+  return RATP_OK;
 }
 
 }  // extern "C"

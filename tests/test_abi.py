@@ -140,6 +140,21 @@ def test_decode_rejects_mismatched_cache_on_host(lib):
                                 ctypes.cast(mask, ctypes.c_void_p), None) == 1
 
 
+def test_decode_layers_rejects_bad_arguments_on_host(lib):
+    assert lib.ratp_decode_step_layers(None, 0, None) == 0
+    assert lib.ratp_decode_step_layers(None, 2, None) == 1
+    arr = (_binding.DecodeLayerStruct * 2)()
+    assert lib.ratp_decode_step_layers(arr, -1, None) == 1
+    # a layer with a NULL field stops the call before any launch
+    assert lib.ratp_decode_step_layers(arr, 2, None) == 1
+
+
+def test_decode_layer_struct_matches_header():
+    src = open(HEADER).read()
+    body = re.search(r"typedef struct ratp_decode_layer \{(.*?)\} ratp_decode_layer;", src, re.S).group(1)
+    assert _struct_fields(body) == [f[0] for f in _binding.DecodeLayerStruct._fields_]
+
+
 def test_missing_library_fails_loudly(tmp_path):
     saved = _binding._lib
     _binding._lib = None
