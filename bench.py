@@ -397,6 +397,49 @@ def measure_chunk_local(name, L_list, dev, steps, warmup, peaks):
     return out
 
 
+def measure_per_sample(name, dev, steps, warmup, peaks):
+    """Prefill of one workload with one dilation per sample in one attention
+    launch: the first half of the batch dense (D = 1), the second half at
+    D = 64 (the batch composition of active recurrence learning).  Timed
+    with CUDA events on the launching stream; reported beside the headline
+    line."""
+    import recurrence_augmented_dilated_chunked_b200 as ratp
+    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
+    w = WORKLOADS[name]
+    Ds = [1] * (w.B // 2) + [64] * (w.B - w.B // 2)
+    stream = torch.cuda.current_stream(dev)
+    q, xk, xv, g = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.H, w.Dh, w.dtype,
+                                                        w.gate_mean, w.gate_std, seed=0))
+    hk, hv, o = (torch.empty_like(q) for _ in range(3))
+    ws = ratp.scan_workspace(w.B, w.T, w.H, w.Dh, q.dtype, dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for i in range(warmup + steps):
+        ev = evs[i - warmup] if i >= warmup else None
+        if ev:
+            ev[0].record(stream)
+        ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, workspace=ws)
+        if ev:
+            ev[1].record(stream)
+        ratp.dilated_attn_prefill_per_sample(q, hk, hv, Ds, 0, out=o)
+        if ev:
+            ev[2].record(stream)
+    torch.cuda.synchronize()
+    ratp.last_error(dev)
+    scan_ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+    attn_ms = statistics.median(e[1].elapsed_time(e[2]) for e in evs)
+    pairs = sum(w.H * attention_pairs(w.T, d, 0) for d in Ds)
+    flops = 4 * w.Dh * pairs
+    E = w.B * w.T * w.H * w.Dh
+    attn_gbs = 4 * E * 2 / (attn_ms / 1e3) / 1e9
+    tfs = flops / (attn_ms / 1e3) / 1e12
+    del q, xk, xv, g, hk, hv, o, ws
+    return {"workload": name, "D_per_sample": Ds, "B": w.B, "T": w.T, "H": w.H, "Dh": w.Dh,
+            "prefill_tokens_per_s": w.B * w.T / ((scan_ms + attn_ms) / 1e3),
+            "scan_ms": scan_ms, "attn_ms": attn_ms, "attn_pairs": pairs, "attn_flops": flops,
+            "attn_tflops": tfs, "attn_frac_tensor": tfs / peaks["bf16_tflops"],
+            "attn_frac_hbm": attn_gbs / peaks["hbm_gbs"]}
+
+
 # A 1.5B-like stack of 24 sequence mixers for the layer-wise hybrid: dense
 # layers at 0 (input) and 12 (middle), every other layer at D = 64 with a
 # 128-token window; decode from 32K-token contexts, 16 sequences.
@@ -704,6 +747,8 @@ def run_ours(args, rank, world, local_rank):
         line["chunk_local_scan"] = measure_chunk_local(PREFILL, [wp.D, 1000], dev,
                                                        min(args.steps, 5), args.warmup, peaks)
         line["layer_stack_decode"] = measure_layer_stack(dev, min(args.steps, 5), args.warmup, peaks)
+        line["per_sample_prefill"] = measure_per_sample("bf16_1p5b_T4096_D16", dev, min(args.steps, 5),
+                                                        args.warmup, peaks)
     if not args.no_cpu_baseline and world >= 1:
         line["cpu_baseline"] = oracle_sample()
     print(json.dumps(line), flush=True)

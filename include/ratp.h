@@ -197,6 +197,24 @@ int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv
                                    const uint8_t* head_mask, int dtype, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Per-sample dilation in one launch (the batch composition of the write-up's
+ * section 2.2 "Active Recurrence Learning": in one batch, half the samples
+ * run dense, D = 1, and half dilated, D = 64; forward only).
+ *
+ * o[b] = ratp_dilated_attn_prefill of sample b alone with D = D_per_sample[b]
+ * (same W and head_mask for every sample): a sample with D = 1 is dense in
+ * every head; in the others, heads with head_mask[h] != 0 stay dense.
+ * D_per_sample: host array of B int32 values >= 1, read during the call only.
+ * Tensors as for ratp_dilated_attn_prefill; bf16 with Dh = 128 only.
+ * Errors: ARG (a D < 1, D_per_sample NULL with B > 0, ...), ALIGN,
+ *   SHAPE (B > 1024), UNSUPPORTED (fp32 or Dh = 64, or more than 4 distinct
+ *   values D > 1 in one call).  B, T or H == 0 is a no-op.
+ * ---------------------------------------------------------------------- */
+int ratp_dilated_attn_prefill_per_sample(const void* q, const void* hk, const void* hv, void* o,
+                                         int B, int T, int H, int Dh, const int32_t* D_per_sample,
+                                         int W, const uint8_t* head_mask, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
  * D-compressed KV cache and decode (RAT+ abstract: the KV cache shrinks by D).
  *
  * Layout (all bf16 rows of Dh elements):

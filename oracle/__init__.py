@@ -14,6 +14,8 @@ ctypes.  Each function cites the page passage it follows in the C source:
                     write-up, united with the optional local window.
 * ``attention``   -- softmax attention over the enumerated key sets.
 * ``attention_mask`` -- brute force over an explicit T x T mask.
+* ``attention_per_sample`` -- one dilation per sample (the batch composition
+                    of the write-up's section 2.2), sample by sample.
 * ``cache_row`` / ``ring_row`` / ``cache_pack`` / ``decode_step`` -- the
                     D-compressed cache and one literal decode step.
 
@@ -136,6 +138,30 @@ def attention(q, hk, hv, D: int, W: int, dense_mask=None, rows=None) -> np.ndarr
     o = np.empty((r.shape[0], Dh), dtype=np.float64)
     _load().orc_attention(_p(q), _p(hk), _p(hv), _p(o), B, T, H, Dh, D, W, mp,
                           _p(r, _L), r.shape[0])
+    return o
+
+
+def attention_per_sample(q, hk, hv, D_per_sample, W: int, dense_mask=None, rows=None) -> np.ndarray:
+    """Attention with one dilation per sample (the batch composition of the
+    write-up's section 2.2: part of the batch dense, D = 1, part dilated):
+    sample b is ``attention`` of that sample alone with D = D_per_sample[b].
+
+    rows: optional int array [n, 3] of (b, t, h); then returns [n, Dh].
+    """
+    q, hk, hv = _f64(q), _f64(hk), _f64(hv)
+    B = q.shape[0]
+    ds = [int(d) for d in D_per_sample]
+    assert len(ds) == B and min(ds, default=1) >= 1
+    if rows is None:
+        return np.concatenate([attention(q[b:b + 1], hk[b:b + 1], hv[b:b + 1], ds[b], W, dense_mask)
+                               for b in range(B)], axis=0) if B else np.empty_like(q)
+    r = np.asarray(rows, dtype=np.int64).reshape(-1, 3)
+    o = np.empty((r.shape[0], q.shape[3]), dtype=np.float64)
+    for b in sorted(set(r[:, 0].tolist())):
+        sel = np.nonzero(r[:, 0] == b)[0]
+        rb = r[sel].copy()
+        rb[:, 0] = 0
+        o[sel] = attention(q[b:b + 1], hk[b:b + 1], hv[b:b + 1], ds[b], W, dense_mask, rows=rb)
     return o
 
 

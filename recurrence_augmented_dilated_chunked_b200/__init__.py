@@ -11,6 +11,7 @@ from ._binding import (  # noqa: F401
     KVCache,
     RatpError,
     dilated_attn_prefill,
+    dilated_attn_prefill_per_sample,
     dilated_attn_prefill_simt,
     debug_fault,
     decode_step_layers,

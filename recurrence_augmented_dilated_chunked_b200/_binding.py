@@ -70,6 +70,7 @@ _SIGS = {
     "ratp_scan_prefill_kv_noalloc": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P], _I),
     "ratp_dilated_attn_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_simt": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
+    "ratp_dilated_attn_prefill_per_sample": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I, _P], _I),
     "ratp_cache_bytes": ([_I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)], _I),
     "ratp_cache_init": ([ctypes.POINTER(CacheStruct), _P, _SZ, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ratp_cache_pack": ([ctypes.POINTER(CacheStruct), _P, _P, _I, _P], _I),
@@ -245,6 +246,32 @@ def dilated_attn_prefill(q, hk, hv, D, W=0, head_mask=None, out=None):
 def dilated_attn_prefill_simt(q, hk, hv, D, W=0, head_mask=None, out=None):
     """Same operation on the CUDA-core kernel (fp32/bf16, Dh 64/128)."""
     return _attn("ratp_dilated_attn_prefill_simt", q, hk, hv, D, W, head_mask, out)
+
+
+def dilated_attn_prefill_per_sample(q, hk, hv, D_per_sample, W=0, head_mask=None, out=None):
+    """Dilated attention with one dilation per sample (``D_per_sample``: B
+    ints >= 1; 1 = the sample runs dense) in one launch; bf16, Dh = 128."""
+    lib = load_library()
+    _need(q, "q")
+    _need(hk, "hk", q.dtype)
+    _need(hv, "hv", q.dtype)
+    B, T, H, Dh = q.shape
+    if hk.shape != q.shape or hv.shape != q.shape:
+        raise ValueError("q, hk, hv must have one shape")
+    ds = [int(d) for d in D_per_sample]
+    if len(ds) != B:
+        raise ValueError("D_per_sample must have B = %d entries" % B)
+    dbuf = (ctypes.c_int32 * max(B, 1))(*ds)
+    if out is None:
+        out = torch.empty_like(q)
+    _need(out, "out", q.dtype)
+    mbuf, mp = _mask_buf(head_mask, H)
+    if q.dtype not in _DTYPE:
+        raise ValueError("unsupported dtype %s" % q.dtype)
+    _check("ratp_dilated_attn_prefill_per_sample", lib.ratp_dilated_attn_prefill_per_sample(
+        _ptr(q), _ptr(hk), _ptr(hv), _ptr(out), B, T, H, Dh, ctypes.cast(dbuf, ctypes.c_void_p),
+        int(W), mp, _DTYPE[q.dtype], _stream(q)))
+    return out
 
 
 def last_error(device=None):

@@ -21,9 +21,18 @@
 // a prefix (dilated; dense: s <= t) or a contiguous range (window), applied as
 // bit masks per 32-column chunk.
 //
+// Items are listed segment by segment; a segment is a product set (samples x
+// heads) of one dilation: samples whose D is 1 with every head, the other
+// samples with the dense heads (both dense), then, per dilation D_c > 1 in
+// ascending order, the samples of D_c with the dilated heads.  One dilation
+// for the whole batch (the per-head hybrid) is the case of a single dilated
+// segment; several (per-sample D, the batch composition of the write-up's
+// section 2.2, where half the samples run dense and half at D = 64) take one
+// strided tensor-map pair each.  Within a segment, late query tiles come first.
+//
 // Two CTAs per SM, persistent over items blockIdx.x, +G, +2G, ... (G = grid
-// size = 2 x SMs; items in heavy-first order: dense heads and late query tiles
-// first).  Per CTA, tensor memory holds S (64 columns), two P buffers (bf16
+// size = 2 x SMs; items in heavy-first order: dense segments and late query
+// tiles first).  Per CTA, tensor memory holds S (64 columns), two P buffers (bf16
 // pairs, 32 columns each) and O (128 columns): 256 columns, half an SM's.
 // Because S and P are separate, S = Q K^T of tile n+1 is issued as soon as
 // the softmax has read S of tile n, so the tensor core computes the next
@@ -79,41 +88,61 @@ constexpr uint32_t kColO = 128;    // O: 128 columns
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
+constexpr int kMaxDil = 4;                 // distinct dilations D > 1 in one launch
+constexpr int kMaxSeg = 2 + kMaxDil;
+constexpr int kMaxSamples = 1024;          // batch size with per-sample dilation
+
+// Head sets a segment ranges over
+constexpr int kHeadsDense = 0, kHeadsDil = 1, kHeadsAll = 2;
+
+struct Segment {
+  int begin;        // first item index of the segment
+  int n_b, n_h;     // samples x heads
+  int b_off;        // samples[b_off + i] is sample i; -1: sample i is b = i
+  int8_t heads;     // kHeadsDense / kHeadsDil / kHeadsAll
+  int8_t cls;       // -1: dense; c >= 0: dilation dil_D[c], tensor maps k[c], v[c]
+};
+
+// Strided ("dilated") views of hk and hv, one pair per dilation class: row s
+// of class c is position s * dil_D[c] + dil_D[c] - 1.
+struct DilMaps {
+  CUtensorMap k[kMaxDil];
+  CUtensorMap v[kMaxDil];
+};
+
 struct Params {
   __nv_bfloat16* o;
-  int B, T, H, D, W_eff, NQ;
-  int n_dense, n_dil;
-  int n_items_dense, n_items;
+  int B, T, H, W_eff, NQ;
+  int n_items, n_seg, n_cls;
   float scale_log2;
   int o_align32;          // output base 32-byte aligned (rows are 256 bytes)
+  int dil_D[kMaxDil];
+  Segment seg[kMaxSeg];
   uint8_t dense_list[RATP_MAX_HEADS];
   uint8_t dil_list[RATP_MAX_HEADS];
+  uint16_t samples[kMaxSamples];   // samples grouped by dilation (per-sample mode)
 };
 
 struct Item {
-  int b, h, t0, t_last, Dd, n_win, n_tiles, p_start;
+  int b, h, t0, t_last, Dd, n_win, n_tiles, p_start, cls;
   bool dense;
 };
 
 __device__ __forceinline__ Item make_item(const Params& p, int idx) {
+  int s = 0;
+  while (s + 1 < p.n_seg && idx >= p.seg[s + 1].begin) ++s;
+  const Segment& g = p.seg[s];
   Item it;
-  int per, qi, rem;
-  if (idx < p.n_items_dense) {
-    per = p.B * p.n_dense;
-    qi = idx / per;
-    rem = idx - qi * per;
-    it.b = rem / p.n_dense;
-    it.h = p.dense_list[rem - it.b * p.n_dense];
-    it.dense = true;
-  } else {
-    idx -= p.n_items_dense;
-    per = p.B * p.n_dil;
-    qi = idx / per;
-    rem = idx - qi * per;
-    it.b = rem / p.n_dil;
-    it.h = p.dil_list[rem - it.b * p.n_dil];
-    it.dense = false;
-  }
+  idx -= g.begin;
+  const int per = g.n_b * g.n_h;
+  const int qi = idx / per;
+  const int rem = idx - qi * per;
+  const int bi = rem / g.n_h;
+  const int hi = rem - bi * g.n_h;
+  it.b = g.b_off < 0 ? bi : (int)p.samples[g.b_off + bi];
+  it.h = g.heads == kHeadsDense ? (int)p.dense_list[hi] : g.heads == kHeadsDil ? (int)p.dil_list[hi] : hi;
+  it.cls = g.cls < 0 ? 0 : g.cls;
+  it.dense = g.cls < 0;
   it.t0 = (p.NQ - 1 - qi) * BM;
   it.t_last = min(it.t0 + BM - 1, p.T - 1);
   if (it.dense) {
@@ -122,8 +151,8 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
     it.p_start = 0;
     it.n_tiles = (it.t_last + 1 + BN - 1) / BN;
   } else {
-    it.Dd = p.D;
-    const int n_dil = max(0, it.t_last - p.W_eff + 1) / p.D;   // slots before the last row's window
+    it.Dd = p.dil_D[it.cls];
+    const int n_dil = max(0, it.t_last - p.W_eff + 1) / it.Dd;   // slots before the last row's window
     it.p_start = max(0, it.t0 - p.W_eff + 1);
     it.n_win = (it.t_last - it.p_start + 1 + BN - 1) / BN;
     it.n_tiles = it.n_win + (n_dil + BN - 1) / BN;
@@ -136,8 +165,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             const __grid_constant__ CUtensorMap tm_kpos,
             const __grid_constant__ CUtensorMap tm_vpos,
-            const __grid_constant__ CUtensorMap tm_kdil,
-            const __grid_constant__ CUtensorMap tm_vdil,
+            const __grid_constant__ DilMaps tm_dil,
             const __grid_constant__ Params p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -186,8 +214,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_kpos);
     prefetch_tmap(&tm_vpos);
-    prefetch_tmap(&tm_kdil);
-    prefetch_tmap(&tm_vdil);
+    for (int c = 0; c < p.n_cls; ++c) {
+      prefetch_tmap(&tm_dil.k[c]);
+      prefetch_tmap(&tm_dil.v[c]);
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -213,7 +243,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int row = (j < it.n_win) ? it.p_start + j * BN : (j - it.n_win) * BN;
           if (n >= 2 && !mbar_wait(b_kempty + 8 * st, ((n - 2) >> 1) & 1, s_abort)) { ok = false; break; }
           if (!(blockIdx.x == 0 && (long long)n == g_fault_attn_ktile)) {   // else: planted failure
-            const CUtensorMap* m = pos ? &tm_kpos : &tm_kdil;
+            const CUtensorMap* m = pos ? &tm_kpos : &tm_dil.k[it.cls];
             const uint32_t fb = b_kfull + 8 * st;
             mbar_arrive_expect_tx(fb, kKTile);
             tma_load_4d(sK + st * kKTile, m, fb, 0, it.h, row, it.b);
@@ -228,7 +258,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             ++nq;
           }
           if (n >= 2 && !mbar_wait(b_pvdone + 8 * st, ((n - 2) >> 1) & 1, s_abort)) { ok = false; break; }
-          const CUtensorMap* m = pos ? &tm_vpos : &tm_vdil;
+          const CUtensorMap* m = pos ? &tm_vpos : &tm_dil.v[it.cls];
           const uint32_t fb = b_vfull + 8 * st;
           mbar_arrive_expect_tx(fb, kKTile);
           tma_load_4d(sV + st * kKTile, m, fb, 0, it.h, row, it.b);

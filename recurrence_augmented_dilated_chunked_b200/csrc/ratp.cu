@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <set>
@@ -267,39 +268,94 @@ bool make_map(CUtensorMap* m, const void* base, long long base_elems, int B, lon
   return r == CUDA_SUCCESS;
 }
 
+// Ds: nullable host array of B per-sample dilations (else every sample has D).
 int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
-                   int B, int T, int H, int D, int W, const uint8_t* head_mask,
+                   int B, int T, int H, const int* Ds, int D, int W, const uint8_t* head_mask,
                    cudaStream_t st) {
+  using attn_tc::Segment;
   attn_tc::Params p;
+  memset(&p, 0, sizeof(p));
   p.o = static_cast<__nv_bfloat16*>(o);
-  p.B = B; p.T = T; p.H = H; p.D = D; p.W_eff = W > 0 ? W : 1;
+  p.B = B; p.T = T; p.H = H; p.W_eff = W > 0 ? W : 1;
   p.NQ = (T + attn_tc::BM - 1) / attn_tc::BM;
   unsigned long long bits[RATP_MAX_HEADS / 64];
-  int rc = read_mask(head_mask, H, bits, p.dense_list, &p.n_dense, p.dil_list, &p.n_dil);
+  int n_dense = 0, n_dil = 0;
+  int rc = read_mask(head_mask, H, bits, p.dense_list, &n_dense, p.dil_list, &n_dil);
   if (rc) return rc;
-  p.n_items_dense = B * p.n_dense * p.NQ;
-  p.n_items = B * H * p.NQ;
+  if (Ds != nullptr && B > attn_tc::kMaxSamples) return RATP_ERR_SHAPE;
+  auto D_of = [&](int b) { return Ds != nullptr ? Ds[b] : D; };
+  // dilation classes: the distinct D > 1, ascending (more keys first)
+  for (int b = 0; b < (Ds != nullptr ? B : 1); ++b) {
+    const int d = D_of(b);
+    if (d < 1) return RATP_ERR_ARG;
+    if (d == 1) continue;
+    bool seen = false;
+    for (int c = 0; c < p.n_cls; ++c) seen = seen || p.dil_D[c] == d;
+    if (seen) continue;
+    if (p.n_cls == attn_tc::kMaxDil) return RATP_ERR_UNSUPPORTED;
+    p.dil_D[p.n_cls++] = d;
+  }
+  std::sort(p.dil_D, p.dil_D + p.n_cls);
+  // segments, heavy first: dense, then each dilation class
+  long long items = 0;
+  auto add = [&](int n_b, int b_off, int n_h, int heads, int cls) {
+    if ((long long)n_b * n_h == 0) return;
+    Segment& g = p.seg[p.n_seg++];
+    g.begin = (int)items; g.n_b = n_b; g.n_h = n_h; g.b_off = b_off;
+    g.heads = (int8_t)heads; g.cls = (int8_t)cls;
+    items += (long long)n_b * n_h * p.NQ;
+  };
+  if (Ds == nullptr) {
+    if (D == 1) {
+      add(B, -1, H, attn_tc::kHeadsAll, -1);
+    } else {
+      add(B, -1, n_dense, attn_tc::kHeadsDense, -1);
+      add(B, -1, n_dil, attn_tc::kHeadsDil, 0);
+    }
+  } else {
+    // samples ordered: dense ones, then class 0, class 1, ...
+    int n = 0;
+    for (int b = 0; b < B; ++b) if (D_of(b) == 1) p.samples[n++] = (uint16_t)b;
+    const int n_ds = n;
+    int off[attn_tc::kMaxDil], cnt[attn_tc::kMaxDil];
+    for (int c = 0; c < p.n_cls; ++c) {
+      off[c] = n;
+      for (int b = 0; b < B; ++b) if (D_of(b) == p.dil_D[c]) p.samples[n++] = (uint16_t)b;
+      cnt[c] = n - off[c];
+    }
+    add(n_ds, 0, H, attn_tc::kHeadsAll, -1);
+    add(B - n_ds, n_ds, n_dense, attn_tc::kHeadsDense, -1);
+    for (int c = 0; c < p.n_cls; ++c) add(cnt[c], off[c], n_dil, attn_tc::kHeadsDil, c);
+  }
+  if (items > 0x7fffffffll) return RATP_ERR_SHAPE;
+  p.n_items = (int)items;
+  if (p.n_items == 0) return RATP_OK;
   p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   const long long row = (long long)H * 128, bat = (long long)T * row;
-  CUtensorMap tq, tkp, tvp, tkd, tvd;
+  CUtensorMap tq, tkp, tvp;
+  attn_tc::DilMaps dm;
+  memset(&dm, 0, sizeof(dm));
   constexpr int qr = attn_tc::BM, kr = attn_tc::BN;
   if (!make_map(&tq, q, 0, B, T, H, row, bat, qr) || !make_map(&tkp, hk, 0, B, T, H, row, bat, kr) ||
       !make_map(&tvp, hv, 0, B, T, H, row, bat, kr))
     return RATP_ERR_CUDA;
-  const long long n_slots = T / D;
-  if (n_slots >= 1) {
-    if (!make_map(&tkd, hk, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat, kr) ||
-        !make_map(&tvd, hv, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat, kr))
-      return RATP_ERR_CUDA;
-  } else {
-    tkd = tkp;   // no dilated slot exists for any query: never read
-    tvd = tvp;
+  for (int c = 0; c < attn_tc::kMaxDil; ++c) {
+    const int d = c < p.n_cls ? p.dil_D[c] : 0;
+    const long long n_slots = d > 0 ? T / d : 0;
+    if (n_slots >= 1) {
+      if (!make_map(&dm.k[c], hk, (long long)(d - 1) * row, B, n_slots, H, (long long)d * row, bat, kr) ||
+          !make_map(&dm.v[c], hv, (long long)(d - 1) * row, B, n_slots, H, (long long)d * row, bat, kr))
+        return RATP_ERR_CUDA;
+    } else {
+      dm.k[c] = tkp;   // no dilated slot exists for any query: never read
+      dm.v[c] = tvp;
+    }
   }
   if (!ensure_smem(attn_tc::attn_kernel, (int)attn_tc::kSmemBytes)) return RATP_ERR_CUDA;
   const int slots = attn_tc::kCtasPerSm * sm_count();
   const int grid = p.n_items < slots ? p.n_items : slots;
-  attn_tc::attn_kernel<<<grid, attn_tc::kThreads, attn_tc::kSmemBytes, st>>>(tq, tkp, tvp, tkd, tvd, p);
+  attn_tc::attn_kernel<<<grid, attn_tc::kThreads, attn_tc::kSmemBytes, st>>>(tq, tkp, tvp, dm, p);
   return launch_status();
 }
 
@@ -527,8 +583,23 @@ int ratp_dilated_attn_prefill(const void* q, const void* hk, const void* hv, voi
   if ((long long)B * T * H == 0) return RATP_OK;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (dtype == RATP_BF16 && Dh == 128)
-    return launch_attn_tc(q, hk, hv, o, B, T, H, D, W, head_mask, st);
+    return launch_attn_tc(q, hk, hv, o, B, T, H, nullptr, D, W, head_mask, st);
   return launch_attn_simt(q, hk, hv, o, B, T, H, Dh, D, W, head_mask, dtype, st);
+}
+
+int ratp_dilated_attn_prefill_per_sample(const void* q, const void* hk, const void* hv, void* o,
+                                         int B, int T, int H, int Dh, const int32_t* D_per_sample,
+                                         int W, const uint8_t* head_mask, int dtype, void* stream) {
+  int rc = check_attn_args(q, hk, hv, o, B, T, H, Dh, 1, W, dtype);
+  if (rc) return rc;
+  if (B > 0 && D_per_sample == nullptr) return RATP_ERR_ARG;
+  for (int b = 0; b < B; ++b)
+    if (D_per_sample[b] < 1) return RATP_ERR_ARG;
+  if (dtype != RATP_BF16 || Dh != 128) return RATP_ERR_UNSUPPORTED;
+  if (B > attn_tc::kMaxSamples) return RATP_ERR_SHAPE;
+  if ((long long)B * T * H == 0) return RATP_OK;
+  return launch_attn_tc(q, hk, hv, o, B, T, H, D_per_sample, 0, W, head_mask,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int ratp_cache_bytes(int B, int H, int Dh, int T_max, int D, int W,

@@ -140,6 +140,23 @@ def test_decode_rejects_mismatched_cache_on_host(lib):
                                 ctypes.cast(mask, ctypes.c_void_p), None) == 1
 
 
+def test_per_sample_attention_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)
+    ds = (ctypes.c_int32 * 4)(1, 64, 0, 1)
+    dp = ctypes.cast(ds, ctypes.c_void_p)
+    assert lib.ratp_dilated_attn_prefill_per_sample(p, p, p, p, 2, 8, 1, 128, None, 0, None, 1, None) == 1
+    assert lib.ratp_dilated_attn_prefill_per_sample(p, p, p, p, 4, 8, 1, 128, dp, 0, None, 1, None) == 1
+    ds[2] = 4
+    assert lib.ratp_dilated_attn_prefill_per_sample(p, p, p, p, 4, 8, 1, 128, dp, 0, None, 0, None) == 7
+    assert lib.ratp_dilated_attn_prefill_per_sample(p, p, p, p, 4, 8, 1, 64, dp, 0, None, 1, None) == 7
+    big = (ctypes.c_int32 * 2000)(*([1] * 2000))
+    assert lib.ratp_dilated_attn_prefill_per_sample(p, p, p, p, 2000, 8, 1, 128,
+                                                    ctypes.cast(big, ctypes.c_void_p), 0, None, 1, None) == 2
+    # empty problem: nothing to do, no launch
+    assert lib.ratp_dilated_attn_prefill_per_sample(None, None, None, None, 4, 0, 1, 128, dp, 0, None, 1,
+                                                    None) == 0
+
+
 def test_decode_layers_rejects_bad_arguments_on_host(lib):
     assert lib.ratp_decode_step_layers(None, 0, None) == 0
     assert lib.ratp_decode_step_layers(None, 2, None) == 1

@@ -10,6 +10,8 @@
 * attention: hand-worked fixture, dense causal attention from
   ``torch.nn.functional.scaled_dot_product_attention`` (fp64) when D = 1 or
   W >= T, the self-only identity when D >= T, and an explicit-mask brute force;
+  per-sample dilation: dense samples equal SDPA, samples with D > T are
+  self-only;
 * cache: hand-worked layout fixture, bijectivity, and prefill/decode
   consistency of the literal decode step.
 """
@@ -194,6 +196,24 @@ def test_attention_dense_heads_are_dense():
     np.testing.assert_allclose(out[:, :, 0], ref[:, :, 0], rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(out[:, :, 2], ref[:, :, 2], rtol=1e-12, atol=1e-12)
     assert not np.allclose(out[:, :, 1], ref[:, :, 1])
+
+
+def test_attention_per_sample_dense_and_self_only_samples():
+    """Samples with D = 1 are dense causal attention (SDPA); samples whose D
+    exceeds the sequence attend only to themselves (o = hv); the others equal
+    the single-dilation attention of their D."""
+    q, k, v = _rand_qkv(4, 23, 2, 8)
+    ds = [1, 30, 4, 1]
+    out = oracle.attention_per_sample(q, k, v, ds, 0)
+    ref = _sdpa_causal(q, k, v)
+    for b in (0, 3):
+        np.testing.assert_allclose(out[b], ref[b], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(out[1], v[1])
+    assert np.array_equal(out[2], oracle.attention(q, k, v, 4, 0)[2])
+    rows = np.array([[2, 22, 1], [0, 5, 0], [1, 7, 1], [2, 3, 0]])
+    got = oracle.attention_per_sample(q, k, v, ds, 0, rows=rows)
+    for i, (b, t, h) in enumerate(rows):
+        assert np.array_equal(got[i], out[b, t, h])
 
 
 def test_attention_dilation_beyond_sequence_is_self():
