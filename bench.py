@@ -531,9 +531,14 @@ def run_ours(args, rank, world, local_rank):
         hk, hv, o = (torch.empty_like(q) for _ in range(3))
         ws = ratp.scan_workspace(w.B, w.T, w.H, w.Dh, q.dtype, dev)
         mask = w.dense_mask if w.dense_heads else None
+        L = w.D if args.variant == "chunk_local" else 0
+        Ds = [1] * (w.B // 2) + [64] * (w.B - w.B // 2)
         for _ in range(args.warmup + args.steps):
-            ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, workspace=ws)
-            ratp.dilated_attn_prefill(q, hk, hv, w.D, w.W, head_mask=mask, out=o)
+            ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, workspace=ws, L=L)
+            if args.variant == "per_sample":
+                ratp.dilated_attn_prefill_per_sample(q, hk, hv, Ds, w.W, head_mask=mask, out=o)
+            else:
+                ratp.dilated_attn_prefill(q, hk, hv, w.D, w.W, head_mask=mask, out=o)
         torch.cuda.synchronize()
         ratp.last_error(dev)
         return 0
@@ -769,6 +774,9 @@ def main():
                     help="run only this part, untimed (a driver for ncu captures)")
     ap.add_argument("--workload", default=None,
                     help="with --only prefill: the prefill workload (default: the headline one)")
+    ap.add_argument("--variant", choices=["chunk_local", "per_sample"], default=None,
+                    help="with --only prefill: chunk-local scan (L = D), or per-sample attention "
+                         "(first half of the batch dense, second half at D = 64)")
     args = ap.parse_args()
     if args.warmup < 3 and args.only is None:
         ap.error("--warmup must be >= 3")
