@@ -469,6 +469,12 @@ def measure_layer_stack(dev, replays, warmup, peaks):
             if W:
                 ring = cache.ring(which)
                 ring.copy_(torch.randn(ring.shape, generator=gen, device=dev, dtype=torch.float32))
+                # a dilated position inside the last W holds one value in both places
+                for h in range(H):
+                    off, _ = cache.head_rows(h)
+                    for pos in range(ctx - W, ctx):
+                        if pos % D == D - 1:
+                            ring[:, h, pos % W] = rows[:, off + pos // D]
         state0 = torch.randn(2, B, H, Dh, generator=gen, device=dev, dtype=torch.float32)
         out = torch.empty(n, B, H, Dh, dtype=torch.bfloat16, device=dev)
         layers.append((cache, state0, state0.clone(), out))

@@ -124,6 +124,7 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   p.epoch = next_scan_epoch();
   p.B = B; p.Tn = Tn; p.C = H * Dh;
   p.reset_L = reset_L;
+  p.l2_ahead = sm_count();   // about one ticket per SM ahead (measured: 100-200 alike)
   p.slabs = geo.slabs; p.n_chains = geo.n_chains; p.n_chunks_t = geo.n_chunks_t;
   const int C = H * Dh, rows = scan::Shape<T>::kChunk;
   CUtensorMap tg, tx0, tx1;

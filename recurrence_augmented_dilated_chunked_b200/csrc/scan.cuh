@@ -22,6 +22,9 @@
 //     epoch-tagged 64-bit words, then reads two predecessors per round trip
 //     and composes their aggregates until it meets an inclusive state.  x and
 //     g are read from HBM exactly once.
+//   * DRAM keeps streaming while CTAs compute: thread 0 of the CTA with ticket
+//     k also prefetches into L2 the tiles of ticket k + l2_ahead (about one
+//     ticket per SM ahead), so the TMA loads of later CTAs mostly hit L2.
 //   * every wait is bounded (spin_timeout()); on expiry the kernel records
 //     RATP_ERR_TIMEOUT, sets a kernel-wide abort word so that no other CTA
 //     keeps waiting, and finishes with a zero carry.
@@ -99,6 +102,12 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
 // Bytes to zero before each launch: the ticket counter.
 inline size_t reset_bytes(long long) { return 256; }
 
+// L2 prefetch of one tile of a 3-D tensor map (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2) : "memory");
+}
+
 __device__ __forceinline__ void put_word(unsigned long long* p, float v, unsigned int epoch) {
   const unsigned long long w = ((unsigned long long)epoch << 32) | __float_as_uint(v);
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(w) : "memory");
@@ -125,6 +134,7 @@ struct Params {
   unsigned int epoch;     // nonzero, unique per launch
   int B, Tn, C;           // Tn tokens, C = H * Dh channels per token
   int reset_L;            // chunk-local block length (RESET kernels only, >= 1)
+  int l2_ahead;           // L2 prefetch distance in tickets (0: none)
   int slabs;              // C / 64
   int n_chains;           // B * slabs
   int n_chunks_t;         // chunks along T
@@ -187,6 +197,18 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     sm100::tma_load_3d(dst, &tm_g, bar, slab * kSlab, chunk * L, b);
     sm100::tma_load_3d(dst + SM::kTile, &tm_x0, bar, slab * kSlab, chunk * L, b);
     if (NS == 2) sm100::tma_load_3d(dst + 2 * SM::kTile, &tm_x1, bar, slab * kSlab, chunk * L, b);
+    // warm L2 with the tiles of the chunk l2_ahead tickets later, so that
+    // DRAM keeps streaming while the resident CTAs compute
+    {
+      const long long nt = (long long)ticket + p.l2_ahead;
+      if (p.l2_ahead > 0 && nt < (long long)p.n_chains * p.n_chunks_t) {
+        const int ck = (int)(nt / p.n_chains), chn = (int)(nt % p.n_chains);
+        const int b2 = chn / p.slabs, s2 = chn % p.slabs;
+        tma_prefetch_l2_3d(&tm_g, s2 * kSlab, ck * L, b2);
+        tma_prefetch_l2_3d(&tm_x0, s2 * kSlab, ck * L, b2);
+        if (NS == 2) tma_prefetch_l2_3d(&tm_x1, s2 * kSlab, ck * L, b2);
+      }
+    }
   }
 
   const int lane_c = tid % LANES;            // 16-byte column within the slab

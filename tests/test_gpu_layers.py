@@ -98,3 +98,76 @@ def test_layer_stack_equals_per_layer_calls_bit_exact():
     for (ca, sa, _, _), (cb, sb, _, _) in zip(a, b):
         assert bits_equal(sa, sb)
         assert bits_equal(ca.lengths(), cb.lengths())
+
+
+def test_layer_stack_full_size_sampled():
+    """The 24-layer layer-wise hybrid at full size (dense layers 0 and 12, the
+    others D = 64 with W = 128; B = 16, H = 16, 32K-token contexts): two
+    token steps through one CUDA graph, checked on sampled sequences of a
+    dense and a dilated layer against the oracle, which reads the same cache
+    contents."""
+    n_layers, dense_layers, Bf, Hf, ctx, steps = 24, (0, 12), 16, 16, 32768, 2
+    gen = torch.Generator(DEV).manual_seed(11)
+    q, xk, xv, g = (x.to(DEV) for x in
+                    ratp.decode_inputs(steps, Bf, Hf, DH, "bf16", 2.0, 1.5, seed=12))
+    layers = []
+    for li in range(n_layers):
+        D, W = (1, 0) if li in dense_layers else (64, 128)
+        cache = ratp.KVCache(Bf, Hf, DH, ctx + steps, D, W)
+        for which in ("k", "v"):
+            rows = cache.dil_rows(which)
+            rows.copy_(torch.randn(rows.shape, generator=gen, device=DEV))
+            if W:
+                ring = cache.ring(which)
+                ring.copy_(torch.randn(ring.shape, generator=gen, device=DEV))
+        if W:
+            # a dilated position inside the last W holds one value in both
+            # places, as after a prefill (the ring row repeats the slot)
+            for h in range(Hf):
+                off, _ = cache.head_rows(h)
+                for pos in range(ctx - W, ctx):
+                    if pos % D == D - 1:
+                        for which in ("k", "v"):
+                            cache.ring(which)[:, h, pos % W] = cache.dil_rows(which)[:, off + pos // D]
+        cache.lengths().fill_(ctx)
+        state = torch.randn(2, Bf, Hf, DH, generator=gen, device=DEV)
+        layers.append((cache, state, state.clone(), torch.empty(steps, Bf, Hf, DH, dtype=torch.bfloat16,
+                                                                device=DEV), D, W))
+    # host copies of what the oracle reads (sampled sequences), taken before any step runs
+    bs = torch.tensor([0, 13], device=DEV)
+    snap = {li: (layers[li][0].dil_rows("k")[bs].cpu(), layers[li][0].dil_rows("v")[bs].cpu(),
+                 None if layers[li][5] == 0 else layers[li][0].ring("k")[bs].cpu(),
+                 None if layers[li][5] == 0 else layers[li][0].ring("v")[bs].cpu(),
+                 layers[li][2][:, bs].cpu()) for li in (0, 1, 12, 23)}
+    buf = [torch.empty(Bf, Hf, DH, dtype=torch.bfloat16, device=DEV) for _ in range(4)]
+
+    def token_step(i):
+        ratp.decode_step_layers([(c, buf[0], buf[1], buf[2], buf[3], st, o[i]) for c, st, _, o, _, _ in layers])
+
+    for k, x in enumerate((q, xk, xv, g)):
+        buf[k].copy_(x[0])
+    token_step(0)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        token_step(1)
+    for k, x in enumerate((q, xk, xv, g)):
+        buf[k].copy_(x[1])
+    graph.replay()
+    torch.cuda.synchronize()
+    ratp.last_error()
+    del graph
+    for li, (kc, vc, kw, vw, st0) in snap.items():
+        cache, _, _, outs, D, W = layers[li]
+        assert cache.lengths().cpu().tolist() == [ctx + steps] * Bf
+        for j, b in enumerate((0, 13)):
+            oc = oracle.Cache(1, Hf, DH, ctx + steps, D, W)
+            oc.Kc[:] = to64(kc[j])
+            oc.Vc[:] = to64(vc[j])
+            if W:
+                oc.Kw[:] = to64(kw[j]).reshape(-1, DH)
+                oc.Vw[:] = to64(vw[j]).reshape(-1, DH)
+            oc.len[:] = ctx
+            oc.state[:] = to64(st0[:, j:j + 1])
+            for i in range(steps):
+                ref = oc.decode_step(*[to64(x[i, b:b + 1].cpu()) for x in (q, xk, xv, g)])
+                assert_close(outs[i, b:b + 1], ref, "bf16", "layer %d (D=%d) b=%d step %d" % (li, D, b, i))
