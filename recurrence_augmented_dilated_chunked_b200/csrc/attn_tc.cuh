@@ -86,6 +86,10 @@ constexpr uint32_t kColS = 0;      // S: 64 columns
 constexpr uint32_t kColP = 64;     // P buffer b at 64 + 32 b
 constexpr uint32_t kColO = 128;    // O: 128 columns
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
+// The O rescale and the epilogue run once per item or less often: their
+// loops stay rolled, which keeps the softmax loop's code compact (measured
+// 2% faster than unrolling them).
+constexpr int kColdUnroll = 1;
 static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
 
 constexpr int kMaxDil = 4;                 // distinct dilations D > 1 in one launch
@@ -447,7 +451,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           // O must hold P V of tile n-1 before it is scaled
           if (!warp_all(mbar_wait(b_pvdone + 8 * (pb ^ 1), ((n - 1) >> 1) & 1, s_abort))) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
+#pragma unroll kColdUnroll
           for (int c = 0; c < 4; ++c) {
             uint32_t o32[32];
             tmem_ld32(colO + 32 * c, o32);
@@ -468,7 +472,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_after();
       const float inv = 1.f / l;
       __nv_bfloat16* orow = p.o + (((size_t)it.b * p.T + t) * p.H + it.h) * DH;
-#pragma unroll
+#pragma unroll kColdUnroll
       for (int c = 0; c < 4; ++c) {
         uint32_t o32[32];
         tmem_ld32(colO + 32 * c, o32);
