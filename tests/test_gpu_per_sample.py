@@ -91,3 +91,19 @@ def test_per_sample_full_size_sampled_rows():
                                           [Ds[b]], 0, rows=rows)
         got = o[b, torch.as_tensor(ts, device=DEV), torch.as_tensor(hs, device=DEV)]
         assert_close(got, ref, "bf16", "sampled rows of sample %d (D=%d)" % (b, Ds[b]))
+
+
+def test_per_sample_largest_batch():
+    """1024 samples (the most one launch takes), every sample its own mix of
+    the dilations {1, 2, 3, 64}; 1025 samples are refused."""
+    B, T, H = 1024, 70, 1
+    q, hk, hv = _inputs(B, T, H, seed=99)
+    Ds = [(1, 2, 3, 64)[(b * 7) % 4] for b in range(B)]
+    o = ratp.dilated_attn_prefill_per_sample(q, hk, hv, Ds, 4)
+    ratp.last_error()
+    ref = oracle.attention_per_sample(to64(q.cpu()), to64(hk.cpu()), to64(hv.cpu()), Ds, 4)
+    assert_close(o, ref, "bf16", "1024 samples")
+    q2, hk2, hv2 = _inputs(B + 1, 8, 1, seed=98)
+    with pytest.raises(RatpError) as e:
+        ratp.dilated_attn_prefill_per_sample(q2, hk2, hv2, [1] * (B + 1))
+    assert e.value.code == 2
