@@ -46,10 +46,10 @@ namespace scan {
 
 constexpr int kThreads = 256;
 constexpr int kSlab = 64;   // channels per chain
-#ifndef RATP_SCAN_ROWS
-#define RATP_SCAN_ROWS 8
-#endif
-constexpr int kRows = RATP_SCAN_ROWS;   // tokens per thread
+// Tokens per thread: 8 gives 256-token bf16 chunks (96 KB of tiles, two CTAs
+// per SM); 4 (128-token chunks, four CTAs per SM, twice the look-backs)
+// measured 25% slower.
+constexpr int kRows = 8;
 
 template <typename T, int R = kRows>
 struct Shape {
