@@ -9,7 +9,10 @@ this module only compiles it with gcc and marshals numpy arrays through
 ctypes.  Each function cites the page passage it follows in the C source:
 
 * ``scan``        -- the forget-gate recurrence of the zhichai.net write-up
-                    "RAT+ 深度拆解", section 2.1 (sequential loop).
+                    "RAT+ 深度拆解", section 2.1 (sequential loop); with L,
+                    the chunk-local variant of the original RAT.
+* ``scan_window`` -- the fixed look-back recurrence of the same section
+                    (window of the last L positions), O(T * L) loop.
 * ``key_set``     -- dilated key set of the RAT+ abstract / section 1 of the
                     write-up, united with the optional local window.
 * ``attention``   -- softmax attention over the enumerated key sets.
@@ -57,6 +60,7 @@ def _load():
         lib = ctypes.CDLL(build())
         lib.orc_scan.argtypes = [_D, _D, _D, ctypes.c_long, ctypes.c_long, ctypes.c_long]
         lib.orc_scan_reset.argtypes = [_D, _D, _D] + [ctypes.c_long] * 4
+        lib.orc_scan_window.argtypes = [_D, _D, _D] + [ctypes.c_long] * 4
         lib.orc_scan_step.argtypes = [_D, _D, _D, ctypes.c_long]
         lib.orc_key_set.argtypes = [ctypes.c_long, ctypes.c_long, ctypes.c_long, _L]
         lib.orc_key_set.restype = ctypes.c_long
@@ -112,6 +116,19 @@ def scan(x, g, L: int = 0) -> np.ndarray:
         _load().orc_scan(_p(x), _p(g), _p(h), B, T, C)
     else:
         _load().orc_scan_reset(_p(x), _p(g), _p(h), B, T, C, L)
+    return h
+
+
+def scan_window(x, g, L: int) -> np.ndarray:
+    """Fixed look-back recurrence: h_t runs h = g h + (1 - g) x from zero over
+    positions max(0, t - L + 1) .. t, along axis 1 of [B, T, ...] arrays."""
+    x = _f64(x)
+    g = _f64(g)
+    assert x.shape == g.shape and x.ndim >= 2 and L >= 1
+    B, T = x.shape[0], x.shape[1]
+    C = int(np.prod(x.shape[2:])) if x.ndim > 2 else 1
+    h = np.empty_like(x)
+    _load().orc_scan_window(_p(x), _p(g), _p(h), B, T, C, L)
     return h
 
 

@@ -32,7 +32,10 @@
  *     with RAT+: each token recurs only inside its own block of L tokens):
  *     the state is zeroed before position t whenever t mod L == 0, at
  *     prefill and at decode alike; the key and value streams restart
- *     together.
+ *     together;
+ *   - fixed look-back variant (the window L* = 64 that the same section
+ *     attributes to RAT+ before it moved to the full sequence): h_t is the
+ *     recurrence over the L positions max(0, t-L+1) .. t, started from zero.
  *
  * Parity pins for every function live in the CPU test-suite (closed forms,
  * brute-force masks, dense causal attention from a library routine,
@@ -86,6 +89,31 @@ void orc_scan_reset(const double* x, const double* g, double* h,
                 if (L > 0 && t % L == 0) state = 0.0;    /* a chunk starts at t */
                 state = g[i] * state + (1.0 - g[i]) * x[i];
                 h[i] = state;
+            }
+        }
+    }
+}
+
+/* Fixed look-back recurrence ([zc] section 2.1: an earlier RAT+ design whose
+ * recurrence window is the L tokens up to and including t, L* = 64): h_t is
+ * the recurrence started from zero at position max(0, t-L+1) and run to t.
+ * A plain O(T * L) loop per channel; L >= T gives the full sequence. */
+void orc_scan_window(const double* x, const double* g, double* h,
+                     long B, long T, long C, long L)
+{
+    long b;
+#pragma omp parallel for schedule(static)
+    for (b = 0; b < B; ++b) {
+        for (long c = 0; c < C; ++c) {
+            for (long t = 0; t < T; ++t) {
+                long j0 = t - L + 1;
+                if (j0 < 0) j0 = 0;
+                double state = 0.0;
+                for (long j = j0; j <= t; ++j) {
+                    long i = (b * T + j) * C + c;
+                    state = g[i] * state + (1.0 - g[i]) * x[i];
+                }
+                h[(b * T + t) * C + c] = state;
             }
         }
     }

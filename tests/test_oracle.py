@@ -5,6 +5,9 @@
 * chunk-local recurrence: L = 1 closed form, the constant-gate closed form
   restarted per block, L >= T equal to the full recurrence, blocks equal to
   independent recurrences, and insensitivity to earlier blocks' inputs;
+* fixed look-back recurrence: L = 1 closed form, L >= T equal to the full
+  recurrence, the constant-gate closed form (a truncated geometric sum), and
+  the block decomposition from explicit sums;
 * key sets: hand-worked fixture, an independent membership predicate, and a
   closed-form count;
 * attention: hand-worked fixture, dense causal attention from
@@ -115,6 +118,56 @@ def test_scan_reset_blocks_are_independent(L):
     h2 = oracle.scan(x2, g, L=L)
     assert np.array_equal(h2[:, 2 * L:], h[:, 2 * L:])
     assert not np.array_equal(h2[:, :L], h[:, :L])
+
+
+# ------------------------------------------------- fixed look-back recurrence
+def test_scan_window_one_token_is_input_weighting():
+    x = RNG.standard_normal((2, 19, 3))
+    g = RNG.uniform(0, 1, x.shape)
+    np.testing.assert_allclose(oracle.scan_window(x, g, 1), (1 - g) * x, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("L", [19, 20, 500])
+def test_scan_window_covering_sequence_is_full(L):
+    x = RNG.standard_normal((2, 19, 4))
+    g = RNG.uniform(0, 1, x.shape)
+    assert np.array_equal(oracle.scan_window(x, g, L), oracle.scan(x, g))
+
+
+@pytest.mark.parametrize("L,c", [(4, 0.7), (16, 0.95), (64, 0.9)])
+def test_scan_window_constant_gate_closed_form(L, c):
+    T = 150
+    x = RNG.standard_normal((1, T, 2))
+    h = oracle.scan_window(x, np.full_like(x, c), L)
+    for t in range(T):
+        k = np.arange(min(t + 1, L))
+        ref = ((1 - c) * c ** k[:, None] * x[0, t - k]).sum(axis=0)
+        np.testing.assert_allclose(h[0, t], ref, rtol=1e-12, atol=1e-12)
+    ones = oracle.scan_window(np.ones((1, T, 1)), np.full((1, T, 1), c), L).ravel()
+    np.testing.assert_allclose(ones, 1 - c ** np.minimum(np.arange(T) + 1, L), rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("L", [4, 16])
+def test_scan_window_matches_blocks_and_suffix_form(L):
+    """At the last position of every block of L the window is the block, so
+    the value equals the chunk-local recurrence there; everywhere it equals
+    the block decomposition loc_t + A_t * S(t - L), built here from explicit
+    sums (A: gate product since the block start, S: the previous block's
+    recurrence over positions t-L+1 .. block end)."""
+    B, T, C = 2, 61, 3
+    x = RNG.standard_normal((B, T, C))
+    g = RNG.uniform(0, 1, (B, T, C))
+    h = oracle.scan_window(x, g, L)
+    loc = oracle.scan(x, g, L=L)
+    ends = [t for t in range(T) if t % L == L - 1]
+    assert np.allclose(h[:, ends], loc[:, ends], rtol=1e-12, atol=1e-12)
+    for t in range(T):
+        c0 = (t // L) * L
+        A = np.prod(g[:, c0:t + 1], axis=1)
+        S = np.zeros((B, C))
+        for j in range(max(0, t - L + 1), c0):
+            S += np.prod(g[:, j + 1:c0], axis=1) * (1 - g[:, j]) * x[:, j]
+        np.testing.assert_allclose(h[:, t], loc[:, t] + A * S, rtol=1e-10, atol=1e-12)
 
 
 # ---------------------------------------------------------------- key sets
