@@ -362,11 +362,11 @@ def measure_config(name, dev, steps, warmup, peaks):
     return out
 
 
-def measure_chunk_local(name, L_list, dev, steps, warmup, peaks):
+def measure_scan_variants(name, L_list, window_L, dev, steps, warmup, peaks):
     """The key/value scan of one workload with the chunk-local recurrence (the
-    original RAT's blocks of L tokens) beside the full-sequence scan, timed
-    with CUDA events on the launching stream.  Reported beside the headline
-    line, not part of it."""
+    original RAT's blocks of L tokens) and with the fixed look-back window,
+    beside the full-sequence scan, timed with CUDA events on the launching
+    stream.  Reported beside the headline line, not part of it."""
     import recurrence_augmented_dilated_chunked_b200 as ratp
     from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
     w = WORKLOADS[name]
@@ -378,21 +378,28 @@ def measure_chunk_local(name, L_list, dev, steps, warmup, peaks):
     ws = ratp.scan_workspace(w.B, w.T, w.H, w.Dh, xk.dtype, dev)
     pc = prefill_counts(w)
     out = {"workload": name}
-    for L in [0] + list(L_list):
+    runs = [("full_sequence", lambda: ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, final_state=fs,
+                                                          workspace=ws))]
+    for L in L_list:
+        runs.append(("chunk_local_L%d" % L,
+                     lambda L=L: ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, final_state=fs,
+                                                      workspace=ws, L=L)))
+    runs.append(("window_L%d" % window_L,
+                 lambda: ratp.scan_prefill_kv_window(xk, xv, g, window_L, hk=hk, hv=hv)))
+    for key, run in runs:
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
         for i in range(warmup + steps):
             ev = evs[i - warmup] if i >= warmup else None
             if ev:
                 ev[0].record(stream)
-            ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, final_state=fs, workspace=ws, L=L)
+            run()
             if ev:
                 ev[1].record(stream)
         torch.cuda.synchronize()
         ratp.last_error(dev)
         ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
         gbs = pc["scan_bytes"] / (ms / 1e3) / 1e9
-        out["full_sequence" if L == 0 else "L%d" % L] = {"scan_ms": ms, "achieved_gbs": gbs,
-                                                         "frac_hbm": gbs / peaks["hbm_gbs"]}
+        out[key] = {"scan_ms": ms, "achieved_gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]}
     del xk, xv, g, hk, hv, ws
     return out
 
@@ -540,7 +547,10 @@ def run_ours(args, rank, world, local_rank):
         L = w.D if args.variant == "chunk_local" else 0
         Ds = [1] * (w.B // 2) + [64] * (w.B - w.B // 2)
         for _ in range(args.warmup + args.steps):
-            ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, workspace=ws, L=L)
+            if args.variant == "window":
+                ratp.scan_prefill_kv_window(xk, xv, g, 64, hk=hk, hv=hv)
+            else:
+                ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, workspace=ws, L=L)
             if args.variant == "per_sample":
                 ratp.dilated_attn_prefill_per_sample(q, hk, hv, Ds, w.W, head_mask=mask, out=o)
             else:
@@ -755,8 +765,8 @@ def run_ours(args, rank, world, local_rank):
         # the other workloads, measured after the timed region (not part of it)
         line["other_configs"] = {n: measure_config(n, dev, min(args.steps, 5), args.warmup, peaks)
                                  for n in OTHER_CONFIGS}
-        line["chunk_local_scan"] = measure_chunk_local(PREFILL, [wp.D, 1000], dev,
-                                                       min(args.steps, 5), args.warmup, peaks)
+        line["scan_variants"] = measure_scan_variants(PREFILL, [wp.D, 1000], 64, dev,
+                                                      min(args.steps, 5), args.warmup, peaks)
         line["layer_stack_decode"] = measure_layer_stack(dev, min(args.steps, 5), args.warmup, peaks)
         line["per_sample_prefill"] = measure_per_sample("bf16_1p5b_T4096_D16", dev, min(args.steps, 5),
                                                         args.warmup, peaks)
@@ -780,9 +790,10 @@ def main():
                     help="run only this part, untimed (a driver for ncu captures)")
     ap.add_argument("--workload", default=None,
                     help="with --only prefill: the prefill workload (default: the headline one)")
-    ap.add_argument("--variant", choices=["chunk_local", "per_sample"], default=None,
-                    help="with --only prefill: chunk-local scan (L = D), or per-sample attention "
-                         "(first half of the batch dense, second half at D = 64)")
+    ap.add_argument("--variant", choices=["chunk_local", "per_sample", "window"], default=None,
+                    help="with --only prefill: chunk-local scan (L = D), per-sample attention "
+                         "(first half of the batch dense, second half at D = 64), or the "
+                         "fixed look-back scan (L = 64)")
     args = ap.parse_args()
     if args.warmup < 3 and args.only is None:
         ap.error("--warmup must be >= 3")

@@ -142,6 +142,26 @@ int ratp_scan_prefill_kv_chunk_local(const void* xk, const void* xv, const void*
                                      void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Fixed look-back recurrence (section 2.1 of the zhichai.net write-up: the
+ * recurrence window L* = 64 of the RAT+ design before it moved to the full
+ * sequence).  Prefill only.
+ *
+ * h_t = the recurrence h = g h + (1 - g) x started from zero at position
+ * max(0, t - L + 1) and run to t, for the key and value streams with one
+ * gate tensor.  xk, xv, g, hk, hv: [B][T][H][Dh] of dtype (bf16 or fp32),
+ * device pointers, 16-byte aligned; hk, hv are written, nothing else is.
+ * L: 16, 32 or 64 (L >= T gives the full-sequence recurrence).  No
+ * workspace: every 256-token chunk is computed from its own tokens and the
+ * L before it.
+ * Errors: ARG (L < 1, null pointer, negative size, bad dtype), UNSUPPORTED
+ *   (another L), SHAPE (H*Dh not a multiple of 64), ALIGN.  B, T or H == 0
+ *   is a no-op.  There is no decode step for this recurrence.
+ * ---------------------------------------------------------------------- */
+int ratp_scan_prefill_kv_window(const void* xk, const void* xv, const void* g,
+                                void* hk, void* hv, int B, int T, int H, int Dh, int dtype,
+                                int L, void* stream);
+
+/* ------------------------------------------------------------------------
  * Allocation-free variant of ratp_scan_prefill_kv.  The paper has no
  * counterpart: this is a convenience of the library.
  *

@@ -21,6 +21,7 @@ from ._binding import (  # noqa: F401
     scan_prefill,
     scan_prefill_kv,
     scan_prefill_kv_noalloc,
+    scan_prefill_kv_window,
     scan_workspace,
     sm_count,
 )

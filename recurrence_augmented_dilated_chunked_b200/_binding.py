@@ -67,6 +67,7 @@ _SIGS = {
     "ratp_scan_prefill_kv": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "ratp_scan_prefill_chunk_local": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "ratp_scan_prefill_kv_chunk_local": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
+    "ratp_scan_prefill_kv_window": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P], _I),
     "ratp_scan_prefill_kv_noalloc": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P], _I),
     "ratp_dilated_attn_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_simt": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
@@ -200,6 +201,24 @@ def scan_prefill_kv(xk, xv, g, hk=None, hv=None, final_state=None, workspace=Non
         _check("ratp_scan_prefill_kv", lib.ratp_scan_prefill_kv(
             _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(final_state),
             B, T, H, Dh, _DTYPE[xk.dtype], _ptr(ws), ws.numel(), _stream(xk)))
+    return hk, hv
+
+
+def scan_prefill_kv_window(xk, xv, g, L, hk=None, hv=None):
+    """(hk, hv) with the fixed look-back recurrence: h_t runs from zero over the
+    last L positions up to t (L = 16, 32 or 64)."""
+    lib = load_library()
+    _need(xk, "xk")
+    _need(xv, "xv", xk.dtype)
+    _need(g, "g", xk.dtype)
+    B, T, H, Dh = xk.shape
+    hk = torch.empty_like(xk) if hk is None else hk
+    hv = torch.empty_like(xv) if hv is None else hv
+    _need(hk, "hk", xk.dtype)
+    _need(hv, "hv", xk.dtype)
+    _check("ratp_scan_prefill_kv_window", lib.ratp_scan_prefill_kv_window(
+        _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), B, T, H, Dh, _DTYPE[xk.dtype], int(L),
+        _stream(xk)))
     return hk, hv
 
 

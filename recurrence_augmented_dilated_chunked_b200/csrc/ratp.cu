@@ -6,6 +6,7 @@
 //   attn_tc.cuh    tensor-core (TMA + tcgen05) dilated/windowed attention
 //   attn_simt.cuh  CUDA-core attention for fp32 / head dim 64
 //   decode.cuh     cache pack and the fused decode step
+//   window.cuh     fixed look-back recurrence (window of the last L tokens)
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <string.h>
@@ -19,6 +20,7 @@
 #include "ratp.h"
 #include "common.cuh"
 #include "scan.cuh"
+#include "window.cuh"
 #include "sm100.cuh"
 #include "attn_tc.cuh"
 #include "attn_simt.cuh"
@@ -87,14 +89,15 @@ EncodeTiledFn encode_fn();
 
 // [B][T][C] view, box of 64 channels x `rows` tokens x 1 sequence, no swizzle.
 template <typename T>
-bool make_scan_map(CUtensorMap* m, const void* base, int B, int Tn, int C, int rows) {
+bool make_scan_map(CUtensorMap* m, const void* base, int B, int Tn, int C, int rows,
+                   int box_ch = scan::kSlab) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const CUtensorMapDataType dt = sizeof(T) == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
                                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)Tn, (cuuint64_t)B};
   const cuuint64_t strides[2] = {(cuuint64_t)C * sizeof(T), (cuuint64_t)Tn * C * sizeof(T)};
-  const cuuint32_t box[3] = {(cuuint32_t)scan::kSlab, (cuuint32_t)rows, 1};
+  const cuuint32_t box[3] = {(cuuint32_t)box_ch, (cuuint32_t)rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -154,6 +157,29 @@ int launch_scan_ns(int NS, const void* const* x, const void* g, void* const* h, 
 }
 
 // reset_L: 0 = the full-sequence recurrence, >= 1 = chunk-local blocks of reset_L tokens
+template <typename E, int L>
+int launch_window(const void* xk, const void* xv, const void* g, void* hk, void* hv,
+                  int B, int T, int H, int Dh, cudaStream_t st) {
+  window::Params<E> p;
+  p.h[0] = static_cast<E*>(hk);
+  p.h[1] = static_cast<E*>(hv);
+  p.B = B; p.Tn = T; p.C = H * Dh;
+  p.slabs = p.C / window::kCh;
+  p.n_chunks_t = (T + window::kChunk - 1) / window::kChunk;
+  const long long grid = (long long)B * p.slabs * p.n_chunks_t;
+  if (grid > 0x7fffffffll) return RATP_ERR_SHAPE;
+  CUtensorMap tg, tx0, tx1;
+  if (!make_scan_map<E>(&tg, g, B, T, p.C, window::kBox, window::kCh) ||
+      !make_scan_map<E>(&tx0, xk, B, T, p.C, window::kBox, window::kCh) ||
+      !make_scan_map<E>(&tx1, xv, B, T, p.C, window::kBox, window::kCh))
+    return RATP_ERR_CUDA;
+  constexpr int smem = window::Smem<E>::kBytes;
+  auto kernel = window::window_kernel<E, L>;
+  if (!ensure_smem(kernel, smem)) return RATP_ERR_CUDA;
+  kernel<<<(unsigned)grid, window::kThreads, smem, st>>>(tg, tx0, tx1, p);
+  return launch_status();
+}
+
 int scan_common(int NS, const void* const* x, const void* g, void* const* h, float* fs,
                 int B, int T, int H, int Dh, int dtype, int reset_L,
                 void* ws, size_t ws_bytes, void* stream) {
@@ -547,6 +573,33 @@ int ratp_scan_prefill_kv_chunk_local(const void* xk, const void* xv, const void*
   const void* xs[2] = {xk, xv};
   void* hs[2] = {hk, hv};
   return scan_common(2, xs, g, hs, final_state, B, T, H, Dh, dtype, L, workspace, workspace_bytes, stream);
+}
+
+int ratp_scan_prefill_kv_window(const void* xk, const void* xv, const void* g,
+                                void* hk, void* hv, int B, int T, int H, int Dh, int dtype,
+                                int L, void* stream) {
+  if (B < 0 || T < 0 || H < 0 || Dh < 0 || L < 1) return RATP_ERR_ARG;
+  if (dtype != RATP_F32 && dtype != RATP_BF16) return RATP_ERR_ARG;
+  if (L != 16 && L != 32 && L != 64) return RATP_ERR_UNSUPPORTED;
+  const long long C = (long long)H * Dh;
+  if (C % 64 != 0 || C > (1ll << 30)) return RATP_ERR_SHAPE;
+  if ((long long)B * T * C == 0) return RATP_OK;
+  if (!xk || !xv || !g || !hk || !hv) return RATP_ERR_ARG;
+  if (!aligned16(xk) || !aligned16(xv) || !aligned16(g) || !aligned16(hk) || !aligned16(hv))
+    return RATP_ERR_ALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == RATP_BF16) {
+    switch (L) {
+      case 16: return launch_window<__nv_bfloat16, 16>(xk, xv, g, hk, hv, B, T, H, Dh, st);
+      case 32: return launch_window<__nv_bfloat16, 32>(xk, xv, g, hk, hv, B, T, H, Dh, st);
+      default: return launch_window<__nv_bfloat16, 64>(xk, xv, g, hk, hv, B, T, H, Dh, st);
+    }
+  }
+  switch (L) {
+    case 16: return launch_window<float, 16>(xk, xv, g, hk, hv, B, T, H, Dh, st);
+    case 32: return launch_window<float, 32>(xk, xv, g, hk, hv, B, T, H, Dh, st);
+    default: return launch_window<float, 64>(xk, xv, g, hk, hv, B, T, H, Dh, st);
+  }
 }
 
 int ratp_scan_prefill_kv_noalloc(const void* xk, const void* xv, const void* g,

@@ -113,6 +113,16 @@ def test_scan_rejects_bad_arguments_on_host(lib):
     assert lib.ratp_scan_prefill(None, None, None, None, 1, 0, 1, 64, 1, None, 0, None) == 0
 
 
+def test_window_scan_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.ratp_scan_prefill_kv_window(p, p, p, p, p, 1, 8, 1, 64, 1, 0, None) == 1
+    assert lib.ratp_scan_prefill_kv_window(p, p, p, p, p, 1, 8, 1, 64, 1, 48, None) == 7
+    assert lib.ratp_scan_prefill_kv_window(p, p, p, p, p, 1, 8, 1, 32, 1, 64, None) == 2
+    assert lib.ratp_scan_prefill_kv_window(None, p, p, p, p, 1, 8, 1, 64, 1, 64, None) == 1
+    assert lib.ratp_scan_prefill_kv_window(ctypes.c_void_p(8), p, p, p, p, 1, 8, 1, 64, 1, 64, None) == 3
+    assert lib.ratp_scan_prefill_kv_window(None, None, None, None, None, 1, 0, 1, 64, 1, 64, None) == 0
+
+
 def test_chunk_local_rejects_bad_arguments_on_host(lib):
     p = ctypes.c_void_p(16)
     # a negative block length is refused before anything else is looked at
