@@ -164,3 +164,22 @@ def test_empty_problem_launches_nothing(B, T, H):
     o = ratp.dilated_attn_prefill(q, q, q, 4, 8)
     ratp.last_error()
     assert o.shape == q.shape
+
+
+@pytest.mark.parametrize("Dh,dtype", [(128, "bf16"), (64, "bf16"), (64, "f32")])
+@pytest.mark.parametrize("D", [1, 2, 3, 4, 16, 64, "T", "T+5"])
+def test_small_shape_sweep(Dh, dtype, D):
+    """Every combination of T in {1, 2, D-1, D, D+1, 257} and W in {0, 1, 3,
+    D, 128} for one dilation (D = T and D = T + 5 taken per T): the bounds of
+    the key-set split, the window and the ragged query tile."""
+    n = 0
+    for T in sorted({1, 2, 257} | ({D - 1, D, D + 1} if isinstance(D, int) else set()) - {0}):
+        d = T if D == "T" else T + 5 if D == "T+5" else D
+        for W in sorted({0, 1, 3, d, 128}):
+            q, k, v = _qkv(1, T, 2, Dh, dtype, seed=1000 * T + 10 * W + d)
+            o = ratp.dilated_attn_prefill(q.to(DEV), k.to(DEV), v.to(DEV), d, W)
+            ref = oracle.attention(to64(q), to64(k), to64(v), d, W)
+            assert_close(o, ref, dtype, "T=%d D=%d W=%d Dh=%d" % (T, d, W, Dh))
+            n += 1
+    ratp.last_error()
+    assert n >= 10
