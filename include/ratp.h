@@ -53,7 +53,9 @@ typedef enum ratp_status {
   RATP_ERR_CAPACITY = 4,    /* workspace/cache too small, cache full  */
   RATP_ERR_TIMEOUT = 5,     /* a bounded device wait ran out          */
   RATP_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed      */
-  RATP_ERR_UNSUPPORTED = 7  /* dtype/shape combination not built      */
+  RATP_ERR_UNSUPPORTED = 7, /* dtype/shape combination not built      */
+  RATP_ERR_BOUNDS = 8       /* guarded build only: an access outside its
+                               buffer was skipped (ratp_guard_line)    */
 } ratp_status;
 
 typedef enum ratp_dtype { RATP_F32 = 0, RATP_BF16 = 1 } ratp_dtype;
@@ -89,6 +91,22 @@ int ratp_device_sm_count(int* sms);
 enum { RATP_FAULT_NONE = 0, RATP_FAULT_SPIN_LIMIT = 1, RATP_FAULT_SCAN_DROP = 2,
        RATP_FAULT_ATTN_DROP_K = 3 };
 int ratp_debug_fault(int kind, long long arg);
+
+/* ------------------------------------------------------------------------
+ * Guarded debug build (libratp_guarded.so, compiled with -DRATP_GUARDED; a
+ * stand-in for a memory checker).  Every global access a kernel addresses
+ * itself is range-checked against its buffer; an access outside it is
+ * skipped and RATP_ERR_BOUNDS is set in the device error word.
+ * ratp_guard_line: *line receives (and the call clears) the source line of
+ *   the first refused access, 0 if none.  Returns RATP_ERR_UNSUPPORTED (and
+ *   *line = 0) in the normal build, so a caller can tell the builds apart.
+ * ratp_debug_guard_probe: guarded build only; one thread asks for element 4
+ *   of a 4-element device array, which the guard refuses (nothing is
+ *   written): the error word then holds RATP_ERR_BOUNDS.  The normal build
+ *   returns RATP_ERR_UNSUPPORTED and launches nothing.
+ * ---------------------------------------------------------------------- */
+int ratp_guard_line(int* line);
+int ratp_debug_guard_probe(void* stream);
 
 /* ------------------------------------------------------------------------
  * Prefill recurrence (write-up section 2.1).

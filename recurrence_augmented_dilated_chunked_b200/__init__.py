@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
     debug_fault,
     decode_step_layers,
     exported_symbols,
+    guard_line,
     last_error,
     load_library,
     scan_prefill,

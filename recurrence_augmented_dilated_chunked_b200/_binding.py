@@ -13,14 +13,16 @@ import threading
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libratp.so")
+# RATP_LIBRARY may name another build of the same C ABI (the guarded debug
+# build, libratp_guarded.so, for bounds-checked test runs)
+LIB_PATH = os.environ.get("RATP_LIBRARY") or os.path.join(_PKG, "libratp.so")
 MAX_HEADS = 256
 
 RATP_F32, RATP_BF16 = 0, 1
 _DTYPE = {torch.float32: RATP_F32, torch.bfloat16: RATP_BF16}
 
 STATUS = {0: "OK", 1: "ERR_ARG", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_CAPACITY",
-          5: "ERR_TIMEOUT", 6: "ERR_CUDA", 7: "ERR_UNSUPPORTED"}
+          5: "ERR_TIMEOUT", 6: "ERR_CUDA", 7: "ERR_UNSUPPORTED", 8: "ERR_BOUNDS"}
 
 
 class RatpError(RuntimeError):
@@ -62,6 +64,8 @@ _SIGS = {
     "ratp_last_error": ([_P], _I),
     "ratp_device_sm_count": ([ctypes.POINTER(_I)], _I),
     "ratp_debug_fault": ([_I, ctypes.c_longlong], _I),
+    "ratp_guard_line": ([ctypes.POINTER(_I)], _I),
+    "ratp_debug_guard_probe": ([_P], _I),
     "ratp_scan_workspace_bytes": ([_I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "ratp_scan_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
     "ratp_scan_prefill_kv": ([_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _SZ, _P], _I),
@@ -406,3 +410,14 @@ def decode_step_layers(layers):
                                    state.data_ptr(), ctypes.pointer(cache.c), out.data_ptr())
     stream = _stream(layers[0][1]) if n else None
     _check("ratp_decode_step_layers", load_library().ratp_decode_step_layers(arr, n, stream))
+
+
+def guard_line():
+    """(guarded build?, source line of the first refused access or 0); the
+    call clears the recorded line."""
+    n = ctypes.c_int()
+    rc = load_library().ratp_guard_line(ctypes.byref(n))
+    if rc == 7:
+        return False, 0
+    _check("ratp_guard_line", rc)
+    return True, n.value

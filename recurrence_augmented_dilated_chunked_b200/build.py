@@ -17,6 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libratp.so")
+# guarded debug build: every kernel-addressed global access range-checked
+GUARDED_LIB = os.path.join(PKG, "libratp_guarded.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 FLAGS = [
@@ -32,26 +34,30 @@ def _sources():
         [os.path.join(INCLUDE, f) for f in sorted(os.listdir(INCLUDE))]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(s) <= t for s in _sources())
 
 
-def build_library(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC] + FLAGS + list(extra) + ["-o", tmp, os.path.join(CSRC, "ratp.cu")]
+def build_library(force: bool = False, verbose: bool = False, extra=(), guarded: bool = False) -> str:
+    """Compile ``libratp.so`` (or, guarded=True, ``libratp_guarded.so`` with
+    -DRATP_GUARDED) unless it is newer than every source."""
+    lib = GUARDED_LIB if guarded else LIB
+    if not force and up_to_date(lib):
+        return lib
+    tmp = lib + ".tmp%d" % os.getpid()
+    flags = FLAGS + (["-DRATP_GUARDED"] if guarded else [])
+    cmd = [NVCC] + flags + list(extra) + ["-o", tmp, os.path.join(CSRC, "ratp.cu")]
     if verbose:
         print(" ".join(cmd), file=sys.stderr)
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     verbose = "-v" in sys.argv
     extra = ["-Xptxas", "-v"] if "--ptxas" in sys.argv else []
-    print(build_library(force=True, verbose=verbose, extra=extra))
+    print(build_library(force=True, verbose=verbose, extra=extra, guarded="--guarded" in sys.argv))

@@ -55,6 +55,8 @@ attn_simt_kernel(const Params p) {
   const T* vbase = hv + b * bstride + (long long)h * DH;
 
   float qv[EPL], acc[EPL];
+  const long long n_elem = (long long)p.B * bstride;
+  if (!RATP_IN(b * bstride + (long long)t * tstride + (long long)h * DH, DH, n_elem)) return;
   load_lane<T, EPL>(q + b * bstride + (long long)t * tstride + (long long)h * DH, lane, qv);
 #pragma unroll
   for (int i = 0; i < EPL; ++i) { qv[i] *= p.scale_log2; acc[i] = 0.f; }
@@ -62,6 +64,7 @@ attn_simt_kernel(const Params p) {
 
   auto visit = [&](int j) {
     float kf[EPL], vf[EPL];
+    if (!RATP_IN(b * bstride + (long long)j * tstride + (long long)h * DH, DH, n_elem)) return;
     load_lane<T, EPL>(kbase + (long long)j * tstride, lane, kf);
     load_lane<T, EPL>(vbase + (long long)j * tstride, lane, vf);
     float s = 0.f;

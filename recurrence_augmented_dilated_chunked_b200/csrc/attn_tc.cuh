@@ -484,6 +484,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               q[i] = pack_bf16x2(__uint_as_float(o32[16 * v + 2 * i]) * inv, __uint_as_float(o32[16 * v + 2 * i + 1]) * inv);
+            if (!RATP_IN((orow - p.o) + 32 * c + 16 * v, 16, (long long)p.B * p.T * p.H * DH)) continue;
             if (p.o_align32) {                       // one 32-byte store per 16 values
               asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
                            :: "l"(orow + 32 * c + 16 * v), "r"(q[0]), "r"(q[1]), "r"(q[2]), "r"(q[3]),

@@ -16,6 +16,29 @@ __device__ __forceinline__ void raise_error(unsigned int code) {
   atomicOr(&g_error_word, 1u << code);
 }
 
+// Guarded debug build (compiled with -DRATP_GUARDED into libratp_guarded.so):
+// every global access that a kernel addresses itself (TMA boxes are bounded by
+// the hardware) first checks its element range against the buffer's size.
+// An access outside it is skipped, RATP_ERR_BOUNDS is set in the error word
+// and the first failing source line is kept in g_guard_line, so an index
+// error shows up as a status instead of a memory fault.  In the normal build
+// RATP_IN(...) is the constant true and costs nothing.
+#ifdef RATP_GUARDED
+__device__ int g_guard_line;
+__device__ __noinline__ bool guard_fail(int line) {
+  atomicCAS(&g_guard_line, 0, line);
+  raise_error(RATP_ERR_BOUNDS);
+  return false;
+}
+__device__ __forceinline__ bool in_range(long long first, long long count, long long size, int line) {
+  return (first >= 0 && count >= 0 && first + count <= size) ? true : guard_fail(line);
+}
+#define RATP_IN(first, count, size) \
+  ::ratp::in_range((long long)(first), (long long)(count), (long long)(size), __LINE__)
+#else
+#define RATP_IN(first, count, size) true
+#endif
+
 // Bound for every spin-wait (ns of %globaltimer).  A wait that runs out sets
 // RATP_ERR_TIMEOUT and the kernel carries on to a clean exit.  Tests of the
 // failure paths lower it and plant a missing publication (ratp_debug_fault).

@@ -120,6 +120,9 @@ decode_kernel(const Params p) {
 
   if (active) {
     const long long bh = (long long)b * p.H + h;
+    const long long n_tok = (long long)p.B * p.H * DH;              // q, x, g, o elements
+    const long long n_dil = (long long)p.B * p.rows_per_b * DH;     // Kc / Vc elements
+    const long long n_ring = (long long)p.B * p.H * p.W * DH;       // Kw / Vw elements
     const __nv_bfloat16* qrow = p.q + bh * DH;
     const long long cache_row0 = (long long)b * p.rows_per_b + head_offset(p.dense_bits, h, p.T_max, p.D);
 
@@ -127,6 +130,8 @@ decode_kernel(const Params p) {
     if (split == 0) {
       for (int c = tid; c < 2 * DH; c += kThreads) {
         const int s = c / DH, ch = c % DH;
+        if (!RATP_IN(((long long)s * p.B * p.H + bh) * DH + ch, 1, 2 * n_tok) ||
+            !RATP_IN(bh * DH + ch, 1, n_tok)) continue;
         float* st = p.state + ((long long)s * p.B * p.H + bh) * DH + ch;
         const float x = __bfloat162float((s == 0 ? p.xk : p.xv)[bh * DH + ch]);
         const float gg = __bfloat162float(p.g[bh * DH + ch]);
@@ -135,9 +140,9 @@ decode_kernel(const Params p) {
         *st = hn;
         const __nv_bfloat16 hb = __float2bfloat16_rn(hn);
         (s == 0 ? s_self_k : s_self_v)[ch] = __bfloat162float(hb);
-        if (t % Dd == Dd - 1 && app_slot < p.T_max / Dd)
+        if (t % Dd == Dd - 1 && app_slot < p.T_max / Dd && RATP_IN((cache_row0 + app_slot) * DH + ch, 1, n_dil))
           (s == 0 ? p.Kc : p.Vc)[(cache_row0 + app_slot) * DH + ch] = hb;
-        if (p.W > 0)
+        if (p.W > 0 && RATP_IN((bh * p.W + t % p.W) * DH + ch, 1, n_ring))
           (s == 0 ? p.Kw : p.Vw)[(bh * p.W + t % p.W) * DH + ch] = hb;
       }
       if (t % Dd == Dd - 1 && app_slot >= p.T_max / Dd && tid == 0) raise_error(RATP_ERR_CAPACITY);
@@ -151,7 +156,8 @@ decode_kernel(const Params p) {
     const unsigned int sub_mask = (LPK == 32) ? 0xffffffffu : (((1u << LPK) - 1u) << (sub * LPK));
     float qf[8];
     {
-      const uint4 qv = *reinterpret_cast<const uint4*>(qrow + li * 8);
+      const uint4 qv = RATP_IN(bh * DH + li * 8, 8, n_tok) ? *reinterpret_cast<const uint4*>(qrow + li * 8)
+                                                             : make_uint4(0u, 0u, 0u, 0u);
       Elem<__nv_bfloat16>::unpack(qv, qf);
 #pragma unroll
       for (int i = 0; i < 8; ++i) qf[i] *= p.scale_log2;
@@ -174,13 +180,13 @@ decode_kernel(const Params p) {
           if (k < n_slots) {
             kr = p.Kc + (cache_row0 + k) * DH;
             vr = p.Vc + (cache_row0 + k) * DH;
-            use[u] = true;
+            use[u] = RATP_IN((cache_row0 + k) * DH, DH, n_dil);
           } else {
             const int pos = w_lo + (k - n_slots);
             const long long rr = (bh * p.W + pos % p.W) * DH;
             kr = p.Kw + rr;
             vr = p.Vw + rr;
-            use[u] = true;
+            use[u] = RATP_IN(rr, DH, n_ring);
           }
           if (use[u]) {
             kv[u] = __ldcs(reinterpret_cast<const uint4*>(kr + li * 8));
@@ -246,6 +252,8 @@ decode_kernel(const Params p) {
 #pragma unroll
     for (int gi = 0; gi < NG; ++gi) M = fmaxf(M, s_m[gi]);
     const bool single = (n_used == 1);
+    const long long n_part = (long long)p.B * p.H * p.max_splits * (DH + 2);
+    const bool part_ok = single || RATP_IN((bh * p.max_splits + split) * (DH + 2), DH + 2, n_part);
     float* part = p.partial + (bh * p.max_splits + split) * (DH + 2);
     for (int c = tid; c < DH; c += kThreads) {
       float L = 0.f, A = 0.f;
@@ -256,8 +264,8 @@ decode_kernel(const Params p) {
         A = fmaf(s_acc[gi][c], w, A);
       }
       if (single) {
-        p.o[bh * DH + c] = __float2bfloat16_rn(A / L);
-      } else {
+        if (RATP_IN(bh * DH + c, 1, n_tok)) p.o[bh * DH + c] = __float2bfloat16_rn(A / L);
+      } else if (part_ok) {
         __stcg(part + 2 + c, A);
         if (c == 0) { __stcg(part, M); __stcg(part + 1, L); }
       }
@@ -273,9 +281,10 @@ decode_kernel(const Params p) {
       if (s_last) {
         __threadfence();
         const float* pb = p.partial + bh * p.max_splits * (DH + 2);
+        const bool pb_ok = RATP_IN(bh * p.max_splits * (DH + 2), (long long)n_used * (DH + 2), n_part);
         float MM = -INFINITY;
         for (int i = 0; i < n_used; ++i) MM = fmaxf(MM, __ldcg(pb + i * (DH + 2)));
-        for (int c = tid; c < DH; c += kThreads) {
+        for (int c = tid; pb_ok && c < DH; c += kThreads) {
           float L = 0.f, A = 0.f;
           for (int i = 0; i < n_used; ++i) {
             const float mi = __ldcg(pb + i * (DH + 2));
@@ -283,7 +292,7 @@ decode_kernel(const Params p) {
             L = fmaf(__ldcg(pb + i * (DH + 2) + 1), w, L);
             A = fmaf(__ldcg(pb + i * (DH + 2) + 2 + c), w, A);
           }
-          p.o[bh * DH + c] = __float2bfloat16_rn(A / L);
+          if (RATP_IN(bh * DH + c, 1, n_tok)) p.o[bh * DH + c] = __float2bfloat16_rn(A / L);
         }
         if (tid == 0) p.counters[bh] = 0u;
       }
@@ -338,16 +347,19 @@ pack_kernel(const PackParams p) {
   const int n_ring = (p.W > 0) ? (p.T - w_lo) : 0;
   if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) p.len[b] = p.T;
   const long long src_base = (long long)b * p.T * p.H * DH + (long long)h * DH + li * 8;
+  const long long n_src = (long long)p.B * p.T * p.H * DH;
   if (r < n_dil) {
     const int pos = r * Dd + Dd - 1;
     const long long src = src_base + (long long)pos * p.H * DH;
     const long long dst = ((long long)b * p.rows_per_b + head_offset(p.dense_bits, h, p.T_max, p.D) + r) * DH + li * 8;
+    if (!RATP_IN(src, 8, n_src) || !RATP_IN(dst, 8, (long long)p.B * p.rows_per_b * DH)) return;
     *reinterpret_cast<uint4*>(p.Kc + dst) = *reinterpret_cast<const uint4*>(p.hk + src);
     *reinterpret_cast<uint4*>(p.Vc + dst) = *reinterpret_cast<const uint4*>(p.hv + src);
   } else if (r < n_dil + n_ring) {
     const int pos = w_lo + (r - n_dil);
     const long long src = src_base + (long long)pos * p.H * DH;
     const long long dst = (((long long)b * p.H + h) * p.W + pos % p.W) * DH + li * 8;
+    if (!RATP_IN(src, 8, n_src) || !RATP_IN(dst, 8, (long long)p.B * p.H * p.W * DH)) return;
     *reinterpret_cast<uint4*>(p.Kw + dst) = *reinterpret_cast<const uint4*>(p.hk + src);
     *reinterpret_cast<uint4*>(p.Vw + dst) = *reinterpret_cast<const uint4*>(p.hv + src);
   }

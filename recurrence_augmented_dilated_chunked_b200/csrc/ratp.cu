@@ -21,6 +21,18 @@
 #include "common.cuh"
 #include "scan.cuh"
 #include "window.cuh"
+
+#ifdef RATP_GUARDED
+namespace ratp {
+// Self-test of the guard: asks for element 4 of a 4-element array.  The
+// guard refuses it (the store never executes) and records RATP_ERR_BOUNDS.
+__device__ int g_guard_probe_buf[4];
+__global__ void guard_probe_kernel() {
+  const int i = 4;
+  if (RATP_IN(i, 1, 4)) g_guard_probe_buf[i & 3] = 1;
+}
+}  // namespace ratp
+#endif
 #include "sm100.cuh"
 #include "attn_tc.cuh"
 #include "attn_simt.cuh"
@@ -481,6 +493,7 @@ const char* ratp_status_string(int status) {
     case RATP_ERR_TIMEOUT: return "bounded device wait expired";
     case RATP_ERR_CUDA: return "CUDA error";
     case RATP_ERR_UNSUPPORTED: return "unsupported dtype/shape combination";
+    case RATP_ERR_BOUNDS: return "guarded build: an out-of-range access was skipped";
     default: return "unknown status";
   }
 }
@@ -495,6 +508,29 @@ int ratp_last_error(void* stream) {
   for (int code = 1; code < 32; ++code)
     if (word & (1u << code)) return code;
   return RATP_OK;
+}
+
+int ratp_guard_line(int* line) {
+  if (!line) return RATP_ERR_ARG;
+  *line = 0;
+#ifdef RATP_GUARDED
+  if (cudaMemcpyFromSymbol(line, ratp::g_guard_line, sizeof(int)) != cudaSuccess) return RATP_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(ratp::g_guard_line, &zero, sizeof(int)) != cudaSuccess) return RATP_ERR_CUDA;
+  return RATP_OK;
+#else
+  return RATP_ERR_UNSUPPORTED;
+#endif
+}
+
+int ratp_debug_guard_probe(void* stream) {
+#ifdef RATP_GUARDED
+  ratp::guard_probe_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>();
+  return launch_status();
+#else
+  (void)stream;
+  return RATP_ERR_UNSUPPORTED;
+#endif
 }
 
 int ratp_debug_fault(int kind, long long arg) {

@@ -242,7 +242,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     if (!__syncthreads_and(ok)) {
       // give up: publish a zero state for this chunk and make every other
       // CTA stop waiting
-      if (tid < 32) {
+      if (tid < 32 && RATP_IN(desc, 1, (long long)p.n_chains * p.n_chunks_t)) {
 #pragma unroll
         for (int w = 0; w < 2 * NS; ++w)
           put_word(p.ws.incl + (desc * 2 * NS + w) * kDescLanes + tid, 0.f, p.epoch);
@@ -405,7 +405,8 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     float cb0[NS], cb1[NS];
 #pragma unroll
     for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
-    if (chunk > 0 && !drop) {
+    const long long n_desc = (long long)p.n_chains * p.n_chunks_t;
+    if (chunk > 0 && !drop && RATP_IN(desc, 1, n_desc)) {
       unsigned long long* dst = p.ws.agg + desc * WA * kDescLanes + lane;
       put_word(dst + 0 * kDescLanes, s_tot_a[c0], p.epoch);
       put_word(dst + 1 * kDescLanes, s_tot_a[c0 + 1], p.epoch);
@@ -428,7 +429,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const long long d = chain0 + (top - u);
-          const bool exists = (top - u) >= 0;
+          const bool exists = (top - u) >= 0 && RATP_IN(d, 1, n_desc);
 #pragma unroll
           for (int w = 0; w < WI; ++w) wi[u][w] = exists ? get_word(incl + (d * WI + w) * kDescLanes + lane) : 0ull;
 #pragma unroll
@@ -492,7 +493,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
       }
     }
     // publish the inclusive state of this chunk
-    if (!drop) {
+    if (!drop && RATP_IN(desc, 1, n_desc)) {
       unsigned long long* dst = p.ws.incl + desc * (2 * NS) * kDescLanes + lane;
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
@@ -535,8 +536,10 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
 #pragma unroll
         for (int i = 0; i < V2; ++i) hs[s][i] = fma2(gf[i], sub2(hs[s][i], xf[i]), xf[i]);
         const long long off = base + (long long)t * row_stride;
-        __stcs(reinterpret_cast<uint4*>(p.h[s] + off), Elem<T>::pack2(hs[s]));
-        if (t == p.Tn - 1 && p.final_state != nullptr) {
+        if (RATP_IN(off, V, (long long)p.B * p.Tn * p.C))
+          __stcs(reinterpret_cast<uint4*>(p.h[s] + off), Elem<T>::pack2(hs[s]));
+        if (t == p.Tn - 1 && p.final_state != nullptr &&
+            RATP_IN(((long long)s * p.B + b) * p.C + slab * kSlab + lane_c * V, V, (long long)NS * p.B * p.C)) {
           float* fs = p.final_state + ((long long)s * p.B + b) * p.C + slab * kSlab + lane_c * V;
 #pragma unroll
           for (int i = 0; i < V2; ++i) { fs[2 * i] = hs[s][i].x; fs[2 * i + 1] = hs[s][i].y; }

@@ -160,7 +160,9 @@ window_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ 
       const float xj = to_f(sx[(cur + o) * kCh + c]);
       loc = fmaf(gj, loc - xj, xj);
       A *= gj;
-      if (whole || tb + o < p.Tn) put(dst, fmaf(A, S[o], loc));
+      if ((whole || tb + o < p.Tn) &&
+          RATP_IN((dst - p.h[s]), 1, (long long)p.B * p.Tn * p.C))
+        put(dst, fmaf(A, S[o], loc));
       dst += p.C;
     }
   }

@@ -60,6 +60,22 @@ def test_debug_fault_rejects_unknown_kind_on_host(lib):
 def test_status_strings(lib):
     assert lib.ratp_status_string(0) == b"ok"
     assert b"aligned" in lib.ratp_status_string(3)
+    assert b"guarded" in lib.ratp_status_string(8)
+
+
+def test_normal_build_is_not_guarded(lib):
+    line = ctypes.c_int(-1)
+    assert lib.ratp_guard_line(ctypes.byref(line)) == 7 and line.value == 0
+    assert lib.ratp_debug_guard_probe(None) == 7
+    assert lib.ratp_guard_line(None) == 1
+
+
+def test_guarded_build_exports_the_same_abi():
+    from recurrence_augmented_dilated_chunked_b200 import build as B
+    path = B.build_library(guarded=True)
+    g = ctypes.CDLL(path)
+    for name in _binding.exported_symbols():
+        assert hasattr(g, name), name
 
 
 def test_scan_workspace_query(lib):

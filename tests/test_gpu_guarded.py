@@ -1,0 +1,52 @@
+"""The guarded debug build (libratp_guarded.so: every global access a kernel
+addresses itself is range-checked; an out-of-range access is skipped and
+reported as RATP_ERR_BOUNDS) stands in for a memory checker.  The small GPU
+parity tests run again against it in a child process: any refused access
+raises through ratp.last_error() in those tests and fails them."""
+import os
+import re
+import subprocess
+import sys
+
+import pytest
+
+from recurrence_augmented_dilated_chunked_b200 import build as B
+
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+SMALL_TESTS = ["tests/test_gpu_scan.py", "tests/test_gpu_chunk_local.py", "tests/test_gpu_window.py",
+               "tests/test_gpu_attn.py", "tests/test_gpu_per_sample.py", "tests/test_gpu_decode.py",
+               "tests/test_gpu_layers.py"]
+
+
+def _child(args, timeout):
+    env = dict(os.environ, RATP_LIBRARY=B.build_library(guarded=True))
+    return subprocess.run([sys.executable] + args, cwd=ROOT, env=env, capture_output=True, text=True,
+                          timeout=timeout)
+
+
+def test_guard_refuses_an_out_of_range_access():
+    code = ("import ctypes, recurrence_augmented_dilated_chunked_b200 as r\n"
+            "from recurrence_augmented_dilated_chunked_b200._binding import RatpError\n"
+            "import torch; torch.cuda.init()\n"
+            "lib = r.load_library()\n"
+            "assert r.guard_line() == (True, 0)\n"
+            "assert lib.ratp_debug_guard_probe(None) == 0\n"
+            "try:\n    r.last_error(); raise SystemExit('no error recorded')\n"
+            "except RatpError as e:\n    assert e.code == 8, e.code\n"
+            "guarded, line = r.guard_line()\n"
+            "assert guarded and line > 0, line\n"
+            "print('guard ok', line)\n")
+    res = _child(["-c", code], 300)
+    assert res.returncode == 0, res.stdout + res.stderr
+    assert "guard ok" in res.stdout
+
+
+def test_small_parity_suite_under_the_guarded_build():
+    res = _child(["-m", "pytest", "-x", "-q", "-m", "gpu", "-p", "no:cacheprovider",
+                  "-k", "not full_size and not beyond_2_pow_31 and not largest"] + SMALL_TESTS, 1800)
+    tail = "\n".join((res.stdout + res.stderr).splitlines()[-30:])
+    assert res.returncode == 0, tail
+    m = re.search(r"(\d+) passed", res.stdout)
+    assert m and int(m.group(1)) >= 200, tail
