@@ -173,7 +173,8 @@ int ratp_scan_prefill_kv_chunk_local(const void* xk, const void* xv, const void*
  * L before it.
  * Errors: ARG (L < 1, null pointer, negative size, bad dtype), UNSUPPORTED
  *   (another L), SHAPE (H*Dh not a multiple of 64), ALIGN.  B, T or H == 0
- *   is a no-op.  There is no decode step for this recurrence.
+ *   is a no-op.  Decode continues it through a cache with a window attached
+ *   (ratp_cache_set_window, ratp_cache_pack_inputs).
  * ---------------------------------------------------------------------- */
 int ratp_scan_prefill_kv_window(const void* xk, const void* xv, const void* g,
                                 void* hk, void* hv, int B, int T, int H, int Dh, int dtype,
@@ -277,12 +278,15 @@ typedef struct ratp_cache {
   int32_t* len;
   float* partial;
   uint32_t* counters;
+  void* in_ring;        /* fixed look-back decode: ring of the last window_L inputs,
+                           bf16 [3][B][H][window_L][Dh] (x_k, x_v, g); NULL if unused */
   int64_t rows_per_b;   /* sum_h cap_h */
   int32_t B, H, Dh, T_max, D, W;
   int32_t split_keys;   /* keys per decode split */
   int32_t max_splits;   /* most decode splits any head can need (partial rows per (b, h)) */
   int32_t reset_L;      /* chunk-local recurrence block (0 = full sequence); set by
                            ratp_cache_set_chunk_local */
+  int32_t window_L;     /* fixed look-back window (0 = none); set by ratp_cache_set_window */
   uint8_t dense[RATP_MAX_HEADS];
 } ratp_cache;
 
@@ -307,8 +311,30 @@ int ratp_cache_pack(ratp_cache* c, const void* hk, const void* hv, int T, void* 
  * default that ratp_cache_init sets) is the full-sequence recurrence; L >= 1
  * is the chunk-local recurrence of ratp_scan_prefill_kv_chunk_local, whose
  * state restarts at every position t with t mod L == 0.  Host-only: writes
- * c->reset_L and launches nothing.  Errors: ARG (null c, L < 0). */
+ * c->reset_L and launches nothing.  Errors: ARG (null c, L < 0, or L > 0
+ * with a look-back window attached). */
 int ratp_cache_set_chunk_local(ratp_cache* c, int L);
+
+/* Decode of the fixed look-back recurrence (ratp_scan_prefill_kv_window): the
+ * step needs the inputs of the last L positions, kept in a caller-owned ring.
+ * ratp_cache_window_bytes: bytes of that ring, 3 * B * H * L * Dh bf16
+ *   (x_k, x_v, g; position p in slot p mod L).
+ * ratp_cache_set_window: attaches `ring` (device, >= the bytes above,
+ *   16-byte aligned) and L (1 <= L <= 256) to the cache; L == 0 detaches.
+ *   Host-only.  A cache cannot be both chunk-local and look-back (ARG).
+ * ratp_cache_pack_inputs: prefill -> decode hand-off of the inputs: copies
+ *   positions max(0, T-L) .. T-1 of xk, xv, g (bf16 [B][T][H][Dh], device)
+ *   into the ring (T <= T_max; call after ratp_cache_pack with the same T).
+ * With a window attached, ratp_decode_step first writes the step's inputs
+ * into slot t mod L, then computes the new recurrent key/value as the
+ * recurrence from zero over positions max(0, t-L+1) .. t read from the ring
+ * (O(L) per channel, in split 0) instead of the one-step update; it also
+ * stores that value in `state`.
+ * Errors: ARG, ALIGN, CAPACITY (ring too small, T > T_max). */
+int ratp_cache_window_bytes(int B, int H, int Dh, int L, size_t* bytes);
+int ratp_cache_set_window(ratp_cache* c, void* ring, size_t bytes, int L);
+int ratp_cache_pack_inputs(ratp_cache* c, const void* xk, const void* xv, const void* g, int T,
+                           void* stream);
 
 /* One decode token for every sequence (fused): state <- g*state + (1-g)*x for
  * the key and value streams (fp32 state [2][B][H][Dh], in/out; the state is

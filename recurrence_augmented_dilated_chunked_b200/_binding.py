@@ -37,11 +37,12 @@ class CacheStruct(ctypes.Structure):
         ("Kc", ctypes.c_void_p), ("Vc", ctypes.c_void_p),
         ("Kw", ctypes.c_void_p), ("Vw", ctypes.c_void_p),
         ("len", ctypes.c_void_p), ("partial", ctypes.c_void_p), ("counters", ctypes.c_void_p),
+        ("in_ring", ctypes.c_void_p),
         ("rows_per_b", ctypes.c_int64),
         ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("Dh", ctypes.c_int32),
         ("T_max", ctypes.c_int32), ("D", ctypes.c_int32), ("W", ctypes.c_int32),
         ("split_keys", ctypes.c_int32), ("max_splits", ctypes.c_int32),
-        ("reset_L", ctypes.c_int32),
+        ("reset_L", ctypes.c_int32), ("window_L", ctypes.c_int32),
         ("dense", ctypes.c_uint8 * MAX_HEADS),
     ]
 
@@ -80,6 +81,9 @@ _SIGS = {
     "ratp_cache_init": ([ctypes.POINTER(CacheStruct), _P, _SZ, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ratp_cache_pack": ([ctypes.POINTER(CacheStruct), _P, _P, _I, _P], _I),
     "ratp_cache_set_chunk_local": ([ctypes.POINTER(CacheStruct), _I], _I),
+    "ratp_cache_window_bytes": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "ratp_cache_set_window": ([ctypes.POINTER(CacheStruct), _P, _SZ, _I], _I),
+    "ratp_cache_pack_inputs": ([ctypes.POINTER(CacheStruct), _P, _P, _P, _I, _P], _I),
     "ratp_decode_step": ([_P, _P, _P, _P, _P, ctypes.POINTER(CacheStruct), _P, _I, _I, _P, _P], _I),
     "ratp_decode_step_layers": ([ctypes.POINTER(DecodeLayerStruct), _I, _P], _I),
 }
@@ -376,6 +380,25 @@ class KVCache:
         T = hk.shape[1] if T is None else T
         _check("ratp_cache_pack", load_library().ratp_cache_pack(
             ctypes.byref(self.c), _ptr(hk), _ptr(hv), int(T), _stream(hk)))
+
+    def attach_window(self, L):
+        """Continue a fixed look-back recurrence of window L at decode: keeps a
+        ring of the last L inputs (x_k, x_v, g) beside the cache."""
+        lib = load_library()
+        n = ctypes.c_size_t()
+        _check("ratp_cache_window_bytes",
+               lib.ratp_cache_window_bytes(self.B, self.H, self.Dh, int(L), ctypes.byref(n)))
+        self.in_ring = torch.empty(n.value, dtype=torch.uint8, device=self.buffer.device)
+        _check("ratp_cache_set_window", lib.ratp_cache_set_window(
+            ctypes.byref(self.c), _ptr(self.in_ring), n.value, int(L)))
+
+    def pack_inputs(self, xk, xv, g, T=None):
+        """Prefill -> decode hand-off of the look-back inputs (last L positions)."""
+        for t, nm in ((xk, "xk"), (xv, "xv"), (g, "g")):
+            _need(t, nm, torch.bfloat16)
+        T = xk.shape[1] if T is None else T
+        _check("ratp_cache_pack_inputs", load_library().ratp_cache_pack_inputs(
+            ctypes.byref(self.c), _ptr(xk), _ptr(xv), _ptr(g), int(T), _stream(xk)))
 
     def decode_step(self, q, xk, xv, g, state, out=None):
         """One token per sequence; state: fp32 [2, B, H, Dh] updated in place."""

@@ -44,6 +44,8 @@ struct Params {
   long long rows_per_b;
   int B, H, D, W, T_max, split_keys, max_splits;
   int reset_L;                  // chunk-local recurrence: state restarts at t mod reset_L == 0; 0 = never
+  int window_L;                 // fixed look-back window (0 = none); inputs ring in in_ring
+  __nv_bfloat16* in_ring;       // [3][B][H][window_L][DH]: x_k, x_v, g of the last window_L positions
   float scale_log2;
   int splits_per_b;             // CTAs per batch item: sum over heads of split_base
   int split_base[RATP_MAX_HEADS + 1];   // first CTA (within a batch item) of each head
@@ -128,6 +130,19 @@ decode_kernel(const Params p) {
 
     // ---- split 0: recurrence step, append, ring write, self key ----
     if (split == 0) {
+      const int WL = p.window_L;
+      const long long n_in = 3ll * p.B * p.H * (long long)WL * DH;    // input-ring elements
+      if (WL > 0) {
+        // this step's inputs into slot t mod WL; the window is then
+        // positions max(0, t - WL + 1) .. t of the ring
+        for (int c = tid; c < 3 * DH; c += kThreads) {
+          const int s3 = c / DH, ch = c % DH;
+          const __nv_bfloat16* src = (s3 == 0 ? p.xk : s3 == 1 ? p.xv : p.g) + bh * DH + ch;
+          const long long dst = (((long long)s3 * p.B * p.H + bh) * WL + t % WL) * DH + ch;
+          if (RATP_IN(dst, 1, n_in) && RATP_IN(bh * DH + ch, 1, n_tok)) p.in_ring[dst] = *src;
+        }
+        __syncthreads();
+      }
       for (int c = tid; c < 2 * DH; c += kThreads) {
         const int s = c / DH, ch = c % DH;
         if (!RATP_IN(((long long)s * p.B * p.H + bh) * DH + ch, 1, 2 * n_tok) ||
@@ -135,8 +150,26 @@ decode_kernel(const Params p) {
         float* st = p.state + ((long long)s * p.B * p.H + bh) * DH + ch;
         const float x = __bfloat162float((s == 0 ? p.xk : p.xv)[bh * DH + ch]);
         const float gg = __bfloat162float(p.g[bh * DH + ch]);
-        const float prev = (p.reset_L > 0 && t % p.reset_L == 0) ? 0.f : *st;
-        const float hn = fmaf(gg, prev - x, x);
+        float hn;
+        if (WL > 0) {
+          // fixed look-back: the recurrence from zero over the window
+          const __nv_bfloat16* rx = p.in_ring + ((long long)s * p.B * p.H + bh) * WL * DH + ch;
+          const __nv_bfloat16* rg = p.in_ring + ((long long)2 * p.B * p.H + bh) * WL * DH + ch;
+          float acc_h = 0.f;
+          const int j0 = max(0, t - WL + 1);
+          if (!RATP_IN(((long long)2 * p.B * p.H + bh) * WL * DH, (long long)WL * DH, n_in)) continue;
+#pragma unroll 4
+          for (int j = j0; j <= t; ++j) {
+            const int slot = j % WL;
+            const float gj = __bfloat162float(rg[(long long)slot * DH]);
+            const float xj = __bfloat162float(rx[(long long)slot * DH]);
+            acc_h = fmaf(gj, acc_h - xj, xj);
+          }
+          hn = acc_h;
+        } else {
+          const float prev = (p.reset_L > 0 && t % p.reset_L == 0) ? 0.f : *st;
+          hn = fmaf(gg, prev - x, x);
+        }
         *st = hn;
         const __nv_bfloat16 hb = __float2bfloat16_rn(hn);
         (s == 0 ? s_self_k : s_self_v)[ch] = __bfloat162float(hb);
@@ -362,6 +395,37 @@ pack_kernel(const PackParams p) {
     if (!RATP_IN(src, 8, n_src) || !RATP_IN(dst, 8, (long long)p.B * p.H * p.W * DH)) return;
     *reinterpret_cast<uint4*>(p.Kw + dst) = *reinterpret_cast<const uint4*>(p.hk + src);
     *reinterpret_cast<uint4*>(p.Vw + dst) = *reinterpret_cast<const uint4*>(p.hv + src);
+  }
+}
+
+// prefill -> decode hand-off of the look-back inputs: positions
+// max(0, T - WL) .. T-1 of x_k, x_v, g into ring slots p mod WL.
+// grid (ceil(rows / rows_per_block), H, B); Dh/8 threads per row.
+struct PackInputsParams {
+  const __nv_bfloat16* x[3];    // x_k, x_v, g: [B][T][H][Dh]
+  __nv_bfloat16* in_ring;       // [3][B][H][WL][Dh]
+  int B, T, H, WL;
+};
+
+template <int DH>
+__global__ void __launch_bounds__(256)
+pack_inputs_kernel(const PackInputsParams p) {
+  constexpr int TPR = DH / 8;
+  constexpr int RPB = 256 / TPR;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int r = blockIdx.x * RPB + threadIdx.x / TPR;
+  const int li = threadIdx.x % TPR;
+  const int lo = max(0, p.T - p.WL);
+  if (r >= p.T - lo) return;
+  const int pos = lo + r;
+  const long long src = (((long long)b * p.T + pos) * p.H + h) * DH + li * 8;
+  const long long n_src = (long long)p.B * p.T * p.H * DH;
+  const long long n_ring = 3ll * p.B * p.H * p.WL * DH;
+#pragma unroll
+  for (int s = 0; s < 3; ++s) {
+    const long long dst = (((long long)s * p.B * p.H + (long long)b * p.H + h) * p.WL + pos % p.WL) * DH + li * 8;
+    if (RATP_IN(src, 8, n_src) && RATP_IN(dst, 8, n_ring))
+      *reinterpret_cast<uint4*>(p.in_ring + dst) = *reinterpret_cast<const uint4*>(p.x[s] + src);
   }
 }
 

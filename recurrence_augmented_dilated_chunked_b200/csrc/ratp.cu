@@ -724,6 +724,8 @@ int ratp_cache_init(ratp_cache* c, void* buffer, size_t bytes, int B, int H, int
   c->split_keys = L.split_keys;
   c->max_splits = L.max_splits;
   c->reset_L = 0;
+  c->window_L = 0;
+  c->in_ring = nullptr;
   for (int h = 0; h < H; ++h) c->dense[h] = (head_mask != nullptr && head_mask[h] != 0) ? 1 : 0;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(c->len, 0, (size_t)B * 4, st) != cudaSuccess) return RATP_ERR_CUDA;
@@ -764,8 +766,55 @@ int ratp_cache_pack(ratp_cache* c, const void* hk, const void* hv, int T, void* 
 
 int ratp_cache_set_chunk_local(ratp_cache* c, int L) {
   if (!c || L < 0) return RATP_ERR_ARG;
+  if (L > 0 && c->window_L > 0) return RATP_ERR_ARG;
   c->reset_L = L;
   return RATP_OK;
+}
+
+int ratp_cache_window_bytes(int B, int H, int Dh, int L, size_t* bytes) {
+  if (!bytes || B < 1 || H < 1 || L < 1 || L > 256) return RATP_ERR_ARG;
+  if (Dh != 128 && Dh != 64) return RATP_ERR_SHAPE;
+  *bytes = (size_t)3 * B * H * L * Dh * 2;
+  return RATP_OK;
+}
+
+int ratp_cache_set_window(ratp_cache* c, void* ring, size_t bytes, int L) {
+  if (!c || L < 0 || L > 256) return RATP_ERR_ARG;
+  if (L == 0) {
+    c->window_L = 0;
+    c->in_ring = nullptr;
+    return RATP_OK;
+  }
+  if (!ring || c->reset_L > 0) return RATP_ERR_ARG;
+  if (!aligned16(ring)) return RATP_ERR_ALIGN;
+  size_t need = 0;
+  int rc = ratp_cache_window_bytes(c->B, c->H, c->Dh, L, &need);
+  if (rc) return rc;
+  if (bytes < need) return RATP_ERR_CAPACITY;
+  c->in_ring = ring;
+  c->window_L = L;
+  return RATP_OK;
+}
+
+int ratp_cache_pack_inputs(ratp_cache* c, const void* xk, const void* xv, const void* g, int T,
+                           void* stream) {
+  if (!c || !xk || !xv || !g || c->window_L <= 0 || !c->in_ring) return RATP_ERR_ARG;
+  if (T < 0 || T > c->T_max) return RATP_ERR_CAPACITY;
+  if (!aligned16(xk) || !aligned16(xv) || !aligned16(g)) return RATP_ERR_ALIGN;
+  if (T == 0) return RATP_OK;
+  decode::PackInputsParams p;
+  p.x[0] = static_cast<const __nv_bfloat16*>(xk);
+  p.x[1] = static_cast<const __nv_bfloat16*>(xv);
+  p.x[2] = static_cast<const __nv_bfloat16*>(g);
+  p.in_ring = static_cast<__nv_bfloat16*>(c->in_ring);
+  p.B = c->B; p.T = T; p.H = c->H; p.WL = c->window_L;
+  const int rows = T < c->window_L ? T : c->window_L;
+  const int rpb = 256 / (c->Dh / 8);
+  dim3 grid((unsigned)((rows + rpb - 1) / rpb), (unsigned)c->H, (unsigned)c->B);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (c->Dh == 128) decode::pack_inputs_kernel<128><<<grid, 256, 0, st>>>(p);
+  else decode::pack_inputs_kernel<64><<<grid, 256, 0, st>>>(p);
+  return launch_status();
 }
 
 }  // extern "C"
@@ -778,7 +827,8 @@ namespace {
 int decode_launch(const void* q, const void* xk, const void* xv, const void* g,
                   float* state, const ratp_cache* c, void* o, cudaStream_t st) {
   if (!q || !xk || !xv || !g || !state || !c || !o) return RATP_ERR_ARG;
-  if (c->reset_L < 0) return RATP_ERR_ARG;
+  if (c->reset_L < 0 || c->window_L < 0 || c->window_L > 256) return RATP_ERR_ARG;
+  if (c->window_L > 0 && (c->in_ring == nullptr || c->reset_L > 0)) return RATP_ERR_ARG;
   if (!aligned16(q) || !aligned16(xk) || !aligned16(xv) || !aligned16(g) || !aligned16(state) ||
       !aligned16(o))
     return RATP_ERR_ALIGN;
@@ -801,6 +851,8 @@ int decode_launch(const void* q, const void* xk, const void* xv, const void* g,
   p.split_keys = c->split_keys;
   p.max_splits = c->max_splits;
   p.reset_L = c->reset_L;
+  p.window_L = c->window_L;
+  p.in_ring = static_cast<__nv_bfloat16*>(c->in_ring);
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)c->Dh);
   int rc = read_mask(c->dense, c->H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
   if (rc) return rc;

@@ -183,6 +183,25 @@ def test_per_sample_attention_rejects_bad_arguments_on_host(lib):
                                                     None) == 0
 
 
+def test_cache_window_api_on_host(lib):
+    n = ctypes.c_size_t()
+    assert lib.ratp_cache_window_bytes(2, 3, 128, 64, ctypes.byref(n)) == 0
+    assert n.value == 3 * 2 * 3 * 64 * 128 * 2
+    assert lib.ratp_cache_window_bytes(2, 3, 128, 0, ctypes.byref(n)) == 1
+    assert lib.ratp_cache_window_bytes(2, 3, 96, 8, ctypes.byref(n)) == 2
+    c = _binding.CacheStruct()
+    c.B, c.H, c.Dh, c.T_max = 2, 3, 128, 100
+    p = ctypes.c_void_p(16)
+    assert lib.ratp_cache_set_window(ctypes.byref(c), p, 16, 64) == 4       # ring too small
+    assert lib.ratp_cache_set_window(ctypes.byref(c), ctypes.c_void_p(8), 1 << 30, 64) == 3
+    assert lib.ratp_cache_set_window(ctypes.byref(c), p, 1 << 30, 64) == 0 and c.window_L == 64
+    assert lib.ratp_cache_set_chunk_local(ctypes.byref(c), 4) == 1         # exclusive
+    assert lib.ratp_cache_set_window(ctypes.byref(c), None, 0, 0) == 0 and c.window_L == 0
+    assert lib.ratp_cache_set_chunk_local(ctypes.byref(c), 4) == 0
+    assert lib.ratp_cache_set_window(ctypes.byref(c), p, 1 << 30, 64) == 1  # exclusive
+    assert lib.ratp_cache_pack_inputs(ctypes.byref(c), p, p, p, 10, None) == 1  # no window
+
+
 def test_decode_layers_rejects_bad_arguments_on_host(lib):
     assert lib.ratp_decode_step_layers(None, 0, None) == 0
     assert lib.ratp_decode_step_layers(None, 2, None) == 1

@@ -86,3 +86,51 @@ def test_window_full_size_sampled_channels():
                  w.dtype, "hk sampled")
     assert_close(hv.reshape(w.B, w.T, C)[:, :, cols], oracle.scan_window(to64(xv2), to64(g2), 64),
                  w.dtype, "hv sampled")
+
+
+@pytest.mark.parametrize("B,T,n,H,D,W,L,dense", [
+    (2, 200, 40, 2, 4, 0, 64, ()),        # the window crosses from prefill into decode
+    (2, 40, 30, 2, 16, 16, 64, (0,)),     # prefill shorter than the window
+    (1, 300, 20, 4, 64, 128, 16, (1,)),
+    (2, 96, 70, 2, 3, 8, 32, ()),         # decode runs past a full window
+])
+def test_window_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, L, dense):
+    """Look-back prefill of T tokens, hand-off of the cache and of the last L
+    inputs, then n decode steps: every step equals the oracle's prefill
+    attention over the look-back recurrence of all T + n tokens."""
+    Dh = 128
+    N = T + n
+    mask = [1 if h in dense else 0 for h in range(H)]
+    q, xk, xv, g = prefill_inputs(B, N, H, Dh, "bf16", gate_mean=1.0, gate_std=2.0, seed=N + L)
+    pre = [x[:, :T].contiguous().to(DEV) for x in (xk, xv, g)]
+    hk, hv = ratp.scan_prefill_kv_window(*pre, L)
+    cache = ratp.KVCache(B, H, Dh, N, D, W, head_mask=mask)
+    cache.attach_window(L)
+    cache.pack(hk, hv)
+    cache.pack_inputs(*pre)
+    state = torch.zeros(2, B, H, Dh, dtype=torch.float32, device=DEV)
+    outs = [cache.decode_step(*[x[:, T + i].contiguous().to(DEV) for x in (q, xk, xv, g)], state)
+            for i in range(n)]
+    ratp.last_error()
+    rk = oracle.scan_window(to64(xk), to64(g), L)
+    rv = oracle.scan_window(to64(xv), to64(g), L)
+    ref = oracle.attention(to64(q), rk, rv, D, W, dense_mask=mask)
+    for i in range(n):
+        assert_close(outs[i], ref[:, T + i], "bf16", "decode step %d" % i)
+    # the state holds the last recurrent key/value
+    assert_close(state[0], rk[:, N - 1], "f32", "final k state")
+    assert cache.lengths().cpu().tolist() == [N] * B
+
+
+def test_window_decode_argument_errors():
+    cache = ratp.KVCache(1, 1, 128, 16, 4, 0)
+    with pytest.raises(RatpError):
+        cache.attach_window(300)
+    cache.attach_window(8)
+    with pytest.raises(RatpError):                 # chunk-local and look-back exclude each other
+        ratp._binding._check("set", ratp.load_library().ratp_cache_set_chunk_local(
+            ratp._binding.ctypes.byref(cache.c), 4))
+    x = torch.zeros(1, 17, 1, 128, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(RatpError) as e:            # T > T_max
+        cache.pack_inputs(x, x, x)
+    assert e.value.code == 4
