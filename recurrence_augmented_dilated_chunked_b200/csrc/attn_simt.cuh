@@ -55,7 +55,7 @@ attn_simt_kernel(const Params p) {
   const T* vbase = hv + b * bstride + (long long)h * DH;
 
   float qv[EPL], acc[EPL];
-  const long long n_elem = (long long)p.B * bstride;
+  [[maybe_unused]] const long long n_elem = (long long)p.B * bstride;
   if (!RATP_IN(b * bstride + (long long)t * tstride + (long long)h * DH, DH, n_elem)) return;
   load_lane<T, EPL>(q + b * bstride + (long long)t * tstride + (long long)h * DH, lane, qv);
 #pragma unroll

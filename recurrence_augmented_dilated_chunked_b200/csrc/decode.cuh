@@ -122,16 +122,16 @@ decode_kernel(const Params p) {
 
   if (active) {
     const long long bh = (long long)b * p.H + h;
-    const long long n_tok = (long long)p.B * p.H * DH;              // q, x, g, o elements
-    const long long n_dil = (long long)p.B * p.rows_per_b * DH;     // Kc / Vc elements
-    const long long n_ring = (long long)p.B * p.H * p.W * DH;       // Kw / Vw elements
+    [[maybe_unused]] const long long n_tok = (long long)p.B * p.H * DH;              // q, x, g, o elements
+    [[maybe_unused]] const long long n_dil = (long long)p.B * p.rows_per_b * DH;     // Kc / Vc elements
+    [[maybe_unused]] const long long n_ring = (long long)p.B * p.H * p.W * DH;       // Kw / Vw elements
     const __nv_bfloat16* qrow = p.q + bh * DH;
     const long long cache_row0 = (long long)b * p.rows_per_b + head_offset(p.dense_bits, h, p.T_max, p.D);
 
     // ---- split 0: recurrence step, append, ring write, self key ----
     if (split == 0) {
       const int WL = p.window_L;
-      const long long n_in = 3ll * p.B * p.H * (long long)WL * DH;    // input-ring elements
+      [[maybe_unused]] const long long n_in = 3ll * p.B * p.H * (long long)WL * DH;    // input-ring elements
       if (WL > 0) {
         // this step's inputs into slot t mod WL; the window is then
         // positions max(0, t - WL + 1) .. t of the ring
@@ -285,7 +285,7 @@ decode_kernel(const Params p) {
 #pragma unroll
     for (int gi = 0; gi < NG; ++gi) M = fmaxf(M, s_m[gi]);
     const bool single = (n_used == 1);
-    const long long n_part = (long long)p.B * p.H * p.max_splits * (DH + 2);
+    [[maybe_unused]] const long long n_part = (long long)p.B * p.H * p.max_splits * (DH + 2);
     const bool part_ok = single || RATP_IN((bh * p.max_splits + split) * (DH + 2), DH + 2, n_part);
     float* part = p.partial + (bh * p.max_splits + split) * (DH + 2);
     for (int c = tid; c < DH; c += kThreads) {
@@ -380,7 +380,7 @@ pack_kernel(const PackParams p) {
   const int n_ring = (p.W > 0) ? (p.T - w_lo) : 0;
   if (blockIdx.x == 0 && h == 0 && threadIdx.x == 0) p.len[b] = p.T;
   const long long src_base = (long long)b * p.T * p.H * DH + (long long)h * DH + li * 8;
-  const long long n_src = (long long)p.B * p.T * p.H * DH;
+  [[maybe_unused]] const long long n_src = (long long)p.B * p.T * p.H * DH;
   if (r < n_dil) {
     const int pos = r * Dd + Dd - 1;
     const long long src = src_base + (long long)pos * p.H * DH;
@@ -419,8 +419,8 @@ pack_inputs_kernel(const PackInputsParams p) {
   if (r >= p.T - lo) return;
   const int pos = lo + r;
   const long long src = (((long long)b * p.T + pos) * p.H + h) * DH + li * 8;
-  const long long n_src = (long long)p.B * p.T * p.H * DH;
-  const long long n_ring = 3ll * p.B * p.H * p.WL * DH;
+  [[maybe_unused]] const long long n_src = (long long)p.B * p.T * p.H * DH;
+  [[maybe_unused]] const long long n_ring = 3ll * p.B * p.H * p.WL * DH;
 #pragma unroll
   for (int s = 0; s < 3; ++s) {
     const long long dst = (((long long)s * p.B * p.H + (long long)b * p.H + h) * p.WL + pos % p.WL) * DH + li * 8;

@@ -405,7 +405,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     float cb0[NS], cb1[NS];
 #pragma unroll
     for (int s = 0; s < NS; ++s) { cb0[s] = 0.f; cb1[s] = 0.f; }
-    const long long n_desc = (long long)p.n_chains * p.n_chunks_t;
+    [[maybe_unused]] const long long n_desc = (long long)p.n_chains * p.n_chunks_t;
     if (chunk > 0 && !drop && RATP_IN(desc, 1, n_desc)) {
       unsigned long long* dst = p.ws.agg + desc * WA * kDescLanes + lane;
       put_word(dst + 0 * kDescLanes, s_tot_a[c0], p.epoch);

@@ -198,3 +198,44 @@ def test_hybrid_prefill_then_decode_full_size_sampled():
         t = T + i
         ref = oc.decode_step(*[to64(sl(x)[:, t]) for x in (q, xk, xv, g)])
         assert_close(got[i, b:b + 1], ref, "bf16", "hybrid decode step %d" % i)
+
+
+@pytest.mark.parametrize("D,W,dense", [(4, 8, ()), (16, 0, (1,)), (3, 5, (0,))])
+def test_decode_ragged_lengths(D, W, dense):
+    """Sequences at different positions in one decode launch (len[b] differs):
+    each sequence's prefill is packed on its own and copied into its block of
+    the shared cache; every decode output equals the oracle's prefill
+    attention over that sequence's own tokens."""
+    B, H, Dh, n = 3, 2, 128, 12
+    lens = [250, 131, 7]
+    T_max = max(lens) + n
+    mask = [1 if h in dense else 0 for h in range(H)]
+    cache = ratp.KVCache(B, H, Dh, T_max, D, W, head_mask=mask)
+    state = torch.zeros(2, B, H, Dh, dtype=torch.float32, device=DEV)
+    seqs = []
+    for b, Tb in enumerate(lens):
+        q, xk, xv, g = prefill_inputs(1, Tb + n, H, Dh, "bf16", gate_mean=1.0, gate_std=2.0, seed=70 + b)
+        seqs.append((q, xk, xv, g))
+        fs = torch.zeros(2, 1, H, Dh, dtype=torch.float32, device=DEV)
+        hk, hv = ratp.scan_prefill_kv(xk[:, :Tb].contiguous().to(DEV), xv[:, :Tb].contiguous().to(DEV),
+                                      g[:, :Tb].contiguous().to(DEV), final_state=fs)
+        one = ratp.KVCache(1, H, Dh, T_max, D, W, head_mask=mask)
+        one.pack(hk, hv)
+        for which in ("k", "v"):
+            cache.dil_rows(which)[b].copy_(one.dil_rows(which)[0])
+            if W:
+                cache.ring(which)[b].copy_(one.ring(which)[0])
+        state[:, b] = fs[:, 0]
+    cache.lengths().copy_(torch.tensor(lens, dtype=torch.int32, device=DEV))
+    outs = []
+    for i in range(n):
+        step = [torch.cat([s[k][:, lens[b] + i] for b, s in enumerate(seqs)]).contiguous().to(DEV)
+                for k in range(4)]
+        outs.append(cache.decode_step(*step, state))
+    ratp.last_error()
+    assert cache.lengths().cpu().tolist() == [Tb + n for Tb in lens]
+    for b, (q, xk, xv, g) in enumerate(seqs):
+        rk, rv = oracle.scan(to64(xk), to64(g)), oracle.scan(to64(xv), to64(g))
+        ref = oracle.attention(to64(q), rk, rv, D, W, dense_mask=mask)
+        for i in range(n):
+            assert_close(outs[i][b:b + 1], ref[:, lens[b] + i], "bf16", "b=%d step %d" % (b, i))
