@@ -61,3 +61,40 @@ def test_attention_pair_count_closed_form():
     for T, D, W in [(37, 4, 0), (50, 3, 5), (64, 64, 128), (40, 1, 0), (33, 5, 1)]:
         ref = sum(len(oracle.key_set(t, D, W)) for t in range(T))
         assert bench.attention_pairs(T, D, W) == ref, (T, D, W)
+
+
+def test_decode_bytes_per_step_matches_key_sets():
+    """The decode roofline's algorithmic bytes: every attended cached row once
+    (the oracle's key set minus the token itself), K and V, plus the state,
+    the step's inputs and output, the ring write and the dilated append."""
+    import oracle
+    from recurrence_augmented_dilated_chunked_b200 import Workload
+    for D, W, dense in [(4, 0, ()), (4, 8, ()), (3, 5, (0,)), (64, 128, (1,)), (1, 0, ())]:
+        H, Dh, B = 2, 128, 3
+        w = Workload("t", "bf16", B=B, T=0, H=H, Dh=Dh, D=D, W=W, gate_mean=0.0, gate_std=1.0,
+                     dense_heads=dense)
+        for t in [0, 1, 5, 63, 64, 200, 777]:
+            ref = 0
+            for h in range(H):
+                Dd = 1 if h in dense else D
+                rows = len(oracle.key_set(t, Dd, 0 if Dd == 1 else W)) - 1
+                per = rows * 2 * Dh * 2 + 2 * Dh * 4 * 2 + 4 * Dh * 2 + Dh * 2
+                per += 2 * Dh * 2 if W > 0 else 0
+                per += 2 * Dh * 2 if t % Dd == Dd - 1 else 0
+                ref += B * per
+            assert bench.decode_bytes_per_step(w, t) == ref, (D, W, dense, t)
+
+
+def test_prefill_pair_count_with_dense_heads():
+    import oracle
+    from recurrence_augmented_dilated_chunked_b200 import Workload
+    w = Workload("t", "bf16", B=2, T=45, H=3, Dh=128, D=4, W=6, gate_mean=0.0, gate_std=1.0,
+                 dense_heads=(1,))
+    ref = 0
+    for h in range(3):
+        Dd = 1 if h == 1 else 4
+        ref += 2 * sum(len(oracle.key_set(t, Dd, 0 if Dd == 1 else 6)) for t in range(45))
+    c = bench.prefill_counts(w)
+    assert c["pairs"] == ref
+    assert c["attn_flops"] == 4 * 128 * ref
+    assert c["scan_bytes"] == 5 * 2 * 45 * 3 * 128 * 2
