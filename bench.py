@@ -632,6 +632,10 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     with ClockSampler(dev.index if dev.index is not None else 0) as clk:
         clk.ready()
+        # keep the device busy (~1 ms, before the first event) while the host
+        # queues the first step, so no host-side launch time falls between a
+        # step's events
+        torch.cuda._sleep(2_000_000)
         t_wall = time.perf_counter()
         for i in range(args.steps):
             prefill(evs[i])
