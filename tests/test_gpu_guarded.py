@@ -20,8 +20,14 @@ SMALL_TESTS = ["tests/test_gpu_scan.py", "tests/test_gpu_chunk_local.py", "tests
                "tests/test_gpu_layers.py"]
 
 
+def _env(**extra):
+    env = dict(os.environ, **extra)
+    env["PYTHONPATH"] = ROOT + os.pathsep + env.get("PYTHONPATH", "")
+    return env
+
+
 def _child(args, timeout):
-    env = dict(os.environ, RATP_LIBRARY=B.build_library(guarded=True))
+    env = _env(RATP_LIBRARY=B.build_library(guarded=True))
     return subprocess.run([sys.executable] + args, cwd=ROOT, env=env, capture_output=True, text=True,
                           timeout=timeout)
 
@@ -50,3 +56,43 @@ def test_small_parity_suite_under_the_guarded_build():
     assert res.returncode == 0, tail
     m = re.search(r"(\d+) passed", res.stdout)
     assert m and int(m.group(1)) >= 200, tail
+
+
+_SAME_BITS = r"""
+import sys, torch
+import recurrence_augmented_dilated_chunked_b200 as ratp
+from recurrence_augmented_dilated_chunked_b200 import prefill_inputs
+dev = "cuda"
+B, T, H, Dh, n = 2, 300, 2, 128, 3
+q, xk, xv, g = (x.to(dev) for x in prefill_inputs(B, T + n, H, Dh, "bf16", seed=5))
+pre = [x[:, :T].contiguous() for x in (xk, xv, g)]
+st = torch.zeros(2, B, H, Dh, dtype=torch.float32, device=dev)
+hk, hv = ratp.scan_prefill_kv(*pre, final_state=st)
+o = ratp.dilated_attn_prefill(q[:, :T].contiguous(), hk, hv, 4, 16, head_mask=[1, 0])
+wk, wv = ratp.scan_prefill_kv_window(*pre, 32)
+cache = ratp.KVCache(B, H, Dh, T + n, 4, 16, head_mask=[1, 0])
+cache.pack(hk, hv)
+outs = [cache.decode_step(*[x[:, T + i].contiguous() for x in (q, xk, xv, g)], st) for i in range(n)]
+ratp.last_error()
+torch.save({"hk": hk.cpu(), "o": o.cpu(), "wk": wk.cpu(), "st": st.cpu(),
+            "dec": torch.stack(outs).cpu()}, sys.argv[1])
+"""
+
+
+def test_guarded_build_computes_the_same_bits(tmp_path):
+    """The range checks change no arithmetic: scan, attention, look-back scan
+    and decode give bit-identical results in both builds."""
+    import torch
+    script = tmp_path / "same_bits.py"
+    script.write_text(_SAME_BITS)
+    res = _child([str(script), str(tmp_path / "guarded.pt")], 300)
+    assert res.returncode == 0, res.stdout + res.stderr
+    env = _env()
+    env.pop("RATP_LIBRARY", None)
+    res2 = subprocess.run([sys.executable, str(script), str(tmp_path / "normal.pt")], cwd=ROOT, env=env,
+                          capture_output=True, text=True, timeout=300)
+    assert res2.returncode == 0, res2.stdout + res2.stderr
+    a, b = torch.load(tmp_path / "guarded.pt"), torch.load(tmp_path / "normal.pt")
+    for k in a:
+        assert torch.equal(a[k].view(torch.uint8) if a[k].dtype == torch.bfloat16 else a[k],
+                           b[k].view(torch.uint8) if b[k].dtype == torch.bfloat16 else b[k]), k
