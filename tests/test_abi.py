@@ -225,3 +225,23 @@ def test_missing_library_fails_loudly(tmp_path):
             _binding.load_library(str(tmp_path / "nope.so"))
     finally:
         _binding._lib = saved
+
+
+def test_cpu_tensors_are_refused_not_computed():
+    """There is no CPU path: host tensors are refused before any call."""
+    import torch
+    import recurrence_augmented_dilated_chunked_b200 as ratp
+    x = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16)
+    calls = [
+        lambda: ratp.scan_prefill(x, x),
+        lambda: ratp.scan_prefill_kv(x, x, x),
+        lambda: ratp.scan_prefill_kv(x, x, x, L=4),
+        lambda: ratp.scan_prefill_kv_window(x, x, x, 16),
+        lambda: ratp.scan_prefill_kv_noalloc(x, x, x, x, x),
+        lambda: ratp.dilated_attn_prefill(x, x, x, 4),
+        lambda: ratp.dilated_attn_prefill_simt(x, x, x, 4),
+        lambda: ratp.dilated_attn_prefill_per_sample(x, x, x, [4]),
+    ]
+    for call in calls:
+        with pytest.raises(ValueError):
+            call()
