@@ -8,9 +8,7 @@ the same context computes the right answer.
 """
 import time
 
-import numpy as np
 import pytest
-import torch
 
 import oracle
 import recurrence_augmented_dilated_chunked_b200 as ratp

@@ -7,8 +7,6 @@ These run here on `gloo`, world size 2, with the same calls bench.py makes.
 import os
 import socket
 
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
