@@ -13,7 +13,8 @@ the stream they are launched on; multi-GPU runs are weak-scaled replicas (no
 data-path collective) timed as the max over ranks.
 
 --impl reference times the fp64 CPU oracle (the only executable statement of
-the method there is) on a bounded sample of the same workload.
+the method there is) on the same workload: each step is the whole T=16K
+prefill plus a few literal decode steps of the 32K-context workload.
 """
 from __future__ import annotations
 
@@ -209,71 +210,136 @@ def measured_peaks():
 
 
 # ----------------------------------------------------------------------------- oracle
-def oracle_sample(seconds_target=12.0):
-    """Time the fp64 oracle on a bounded sample of the prefill workload.
+class OracleBaseline:
+    """The fp64 oracle (plain C, OpenMP over rows) on the headline workloads.
 
-    Sample: the scan of both streams over the first `ts` tokens of every
-    sequence (all channels), and attention for `nr` random query rows (b, t, h)
-    of the full-length layer.  Tokens/s = 1 / (scan s/token + attention s/token)
-    where one token is one position of all H heads.
+    prefill(): the whole prefill of the T=16K layer, nothing sampled: the
+    scan of both streams over every token of both sequences and attention of
+    every query row of every head over its key set.
+    decode(n): n literal decode steps (recurrence step, append, attention
+    over the cache contents) for all 64 sequences of the 32K-context
+    workload, continuing from the previous call's position.
+    Inputs are the GPU arm's seeded inputs (rank 0), converted to fp64 once,
+    outside the timed calls, as the GPU arm's inputs are resident in HBM.
     """
-    import oracle
-    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
-    w = WORKLOADS[PREFILL]
-    oracle.build()
-    ts = 1024
-    q, xk, xv, g = prefill_inputs(w.B, ts, w.H, w.Dh, w.dtype, w.gate_mean, w.gate_std, seed=0)
-    x64k, x64v, g64 = (x.to(torch.float64).numpy() for x in (xk, xv, g))
-    t0 = time.perf_counter()
-    oracle.scan(x64k, g64)
-    oracle.scan(x64v, g64)
-    t_scan = (time.perf_counter() - t0) / (w.B * ts)
-    # attention rows: queries from the full-length key sets; keys drawn N(0, 1)
-    rng = np.random.default_rng(0)
-    nr = 2048
-    heads = [0]
-    Tfull = w.T
-    qf, kf, vf, _ = prefill_inputs(1, Tfull, 1, w.Dh, w.dtype, seed=1)
-    rows = np.stack([np.zeros(nr, np.int64), rng.integers(0, Tfull, nr), np.zeros(nr, np.int64)], 1)
-    q64, k64, v64 = (x.to(torch.float64).numpy() for x in (qf, kf, vf))
-    t0 = time.perf_counter()
-    oracle.attention(q64, k64, v64, w.D, w.W, rows=rows)
-    t_attn_row = (time.perf_counter() - t0) / nr
-    t_attn = t_attn_row * w.H
-    tok_s = 1.0 / (t_scan + t_attn)
-    return {"value": tok_s, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": "fp64 oracle: scan of both streams over %d tokens x %d sequences (all %d "
-                      "channels) + attention of %d random query rows of one head at T=%d, D=%d, "
-                      "W=%d; per-token cost = scan + %d heads x row cost" % (
-                          ts, w.B, w.H * w.Dh, nr, Tfull, w.D, w.W, w.H),
-            "scan_s_per_token": t_scan, "attn_s_per_token": t_attn}
+    DECODE_PER_STEP = 4
+
+    def __init__(self):
+        import oracle
+        from recurrence_augmented_dilated_chunked_b200 import (WORKLOADS, decode_context,
+                                                               decode_inputs, prefill_inputs)
+        self.oracle = oracle
+        oracle.build()
+        self.wp, self.wd = WORKLOADS[PREFILL], WORKLOADS[DECODE]
+        w = self.wp
+        self.pre = [x.to(torch.float64).numpy() for x in
+                    prefill_inputs(w.B, w.T, w.H, w.Dh, w.dtype, w.gate_mean, w.gate_std, seed=0)]
+        wd = self.wd
+        steps = wd.decode_steps
+        kd, vd, kw, vw, st0 = decode_context(wd.B, wd.H, wd.Dh, wd.decode_ctx, wd.D, wd.W, seed=2)
+        self.dec_in = [x.to(torch.float64).numpy() for x in
+                       decode_inputs(steps, wd.B, wd.H, wd.Dh, "bf16", wd.gate_mean, wd.gate_std, seed=1)]
+        oc = oracle.Cache(wd.B, wd.H, wd.Dh, wd.decode_ctx + steps, wd.D, wd.W)
+        for b in range(wd.B):
+            for h in range(wd.H):
+                r0 = oracle.cache_row(b, h, 0, wd.H, oc.T_max, wd.D)
+                m = kd[h].shape[1]
+                oc.Kc[r0:r0 + m] = kd[h][b].to(torch.float64).numpy()
+                oc.Vc[r0:r0 + m] = vd[h][b].to(torch.float64).numpy()
+        self.ring0 = (kw.to(torch.float64).numpy().reshape(-1, wd.Dh),
+                      vw.to(torch.float64).numpy().reshape(-1, wd.Dh))
+        self.state0 = st0.to(torch.float64).numpy()
+        self.cache = oc
+        self.pos = steps          # forces a reset on the first decode call
+
+    def prefill(self):
+        q, xk, xv, g = self.pre
+        w = self.wp
+        t0 = time.perf_counter()
+        hk = self.oracle.scan(xk, g)
+        hv = self.oracle.scan(xv, g)
+        self.oracle.attention(q, hk, hv, w.D, w.W)
+        return time.perf_counter() - t0
+
+    def decode(self, n):
+        oc, wd = self.cache, self.wd
+        if self.pos + n > wd.decode_steps:      # back to the start of the context
+            oc.Kw[:], oc.Vw[:] = self.ring0
+            oc.state[:] = self.state0
+            oc.len[:] = wd.decode_ctx
+            self.pos = 0
+        t0 = time.perf_counter()
+        for i in range(self.pos, self.pos + n):
+            oc.decode_step(*[x[i] for x in self.dec_in])
+        self.pos += n
+        return time.perf_counter() - t0
+
+    def describe(self):
+        w, wd = self.wp, self.wd
+        return ("fp64 oracle: the whole prefill of %s (scan of both streams over %d x %d tokens x "
+                "%d channels, attention of all %d query rows x %d heads over their key sets) + "
+                "%d literal decode steps of %s (%d sequences, 32K-token context) per step" % (
+                    PREFILL, w.B, w.T, w.H * w.Dh, w.B * w.T, w.H, self.DECODE_PER_STEP, DECODE, wd.B))
+
+    def measure(self):
+        """One baseline step: (prefill s, decode s) and the derived rates."""
+        t_pre = self.prefill()
+        n = self.DECODE_PER_STEP
+        t_dec = self.decode(n)
+        return t_pre, t_dec
+
+    def summary(self, t_pre, t_dec, cores):
+        w, wd = self.wp, self.wd
+        n = self.DECODE_PER_STEP
+        return {"value": w.B * w.T / t_pre, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                "sample": self.describe(),
+                "prefill": {"tokens_per_s": w.B * w.T / t_pre, "s": t_pre, "cores": cores},
+                "decode": {"tokens_per_s": wd.B * n / t_dec, "s_per_token_step": t_dec / n,
+                           "cores": 1, "steps": n}}
+
+
+def oracle_sample():
+    """The CPU baseline of the GPU line: one baseline step of the oracle."""
+    ob = OracleBaseline()
+    t_pre, t_dec = ob.measure()
+    return ob.summary(t_pre, t_dec, ob.oracle.num_threads())
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
-    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS
-    w = WORKLOADS[PREFILL]
-    vals = []
+    ob = OracleBaseline()
+    cores = ob.oracle.num_threads()
+    pre, dec = [], []
     for i in range(args.warmup + args.steps):
-        r = oracle_sample()
+        t_pre, t_dec = ob.measure()
         if i >= args.warmup:
-            vals.append(r)
-    v = statistics.median([r["value"] for r in vals])
-    tokens = w.B * w.T
+            pre.append(t_pre)
+            dec.append(t_dec)
+    w = ob.wp
+    v = w.B * w.T * args.steps / sum(pre)
+    base = ob.summary(sum(pre) / args.steps, sum(dec) / args.steps, cores)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": tokens / v * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": PREFILL, "B": w.B, "T": w.T, "H": w.H, "Dh": w.Dh, "D": w.D,
-                   "W": w.W},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": vals[0]["cores"],
-                         "kind": "oracle", "sample": vals[0]["sample"]},
+        "ms_per_step": (sum(pre) + sum(dec)) / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": bench_config(w, ob.wd, 1),
+        "prefill": base["prefill"], "decode": base["decode"],
+        "cpu_baseline": base,
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def bench_config(wp, wd, world):
+    """The workload named by the JSON line (both arms)."""
+    return {"workload": PREFILL, "B": wp.B, "T": wp.T, "H": wp.H, "Dh": wp.Dh, "D": wp.D,
+            "W": wp.W, "decode_workload": DECODE, "decode_B": wd.B,
+            "decode_ctx": wd.decode_ctx, "decode_steps": wd.decode_steps,
+            "l2": "no flush: every step streams > 1 GB (inputs larger than L2)",
+            "parallelism": "replicas x%d" % world}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -747,11 +813,7 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": s_total / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": PREFILL, "B": wp.B, "T": wp.T, "H": wp.H, "Dh": wp.Dh, "D": wp.D,
-                   "W": wp.W, "decode_workload": DECODE, "decode_B": wd.B,
-                   "decode_ctx": wd.decode_ctx, "decode_steps": steps,
-                   "l2": "no flush: every step streams > 1 GB (inputs larger than L2)",
-                   "parallelism": "replicas x%d" % world},
+        "config": bench_config(wp, wd, world),
         "prefill": {"tokens_per_s": value, "ms": (s_scan + s_attn) / K},
         "decode": {"tokens_per_s": decode_tok_s, "ms_per_token_step": s_dec / K / steps,
                    "graph": "256 decode launches per CUDA graph"},
@@ -774,7 +836,7 @@ def run_ours(args, rank, world, local_rank):
         line["layer_stack_decode"] = measure_layer_stack(dev, min(args.steps, 5), args.warmup, peaks)
         line["per_sample_prefill"] = measure_per_sample("bf16_1p5b_T4096_D16", dev, min(args.steps, 5),
                                                         args.warmup, peaks)
-    if not args.no_cpu_baseline and world >= 1:
+    if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = oracle_sample()
     print(json.dumps(line), flush=True)
     del graph

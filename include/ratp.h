@@ -122,8 +122,11 @@ int ratp_debug_guard_probe(void* stream);
  *   decode state.
  * workspace: device scratch of at least ratp_scan_workspace_bytes.  It must
  *   be zero-filled once before its first use; every call leaves it valid for
- *   the next one (each launch tags its chunk descriptors with a fresh launch
- *   number), and calls sharing one workspace must be ordered on one stream.
+ *   the next one: each call zeroes its ticket counter on `stream` first, and
+ *   its kernel tags the chunk descriptors with a fresh number kept in the
+ *   workspace itself (so a call replayed from a CUDA graph gets a fresh tag
+ *   as well; tags repeat after 2^32 - 1 calls on one workspace).  Calls
+ *   sharing one workspace must be ordered on one stream.
  *   h may alias x (in-place) only when T == 1.
  * Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of 64), ALIGN,
  *   CAPACITY (workspace too small).  T == 0 or B == 0 is a no-op.
@@ -200,6 +203,9 @@ int ratp_scan_prefill_kv_window(const void* xk, const void* xv, const void* g,
  *     ~53 million elements).
  *   - The first call on a device looks up the array's device address with
  *     that device current; make that first call before any stream capture.
+ *     The address is kept for the life of the process: after
+ *     cudaDeviceReset() on a device this entry point must not be called on
+ *     that device again.
  *   - All calls share the one array, which keeps the previous call's
  *     contents; each call clears, on `stream`, the part that must start at
  *     zero.  Calls that can run at the same time on the GPU (for example on

@@ -146,17 +146,28 @@ def _mask_buf(head_mask, H):
 _ws_cache = {}
 
 
-def scan_workspace(B, T, H, Dh, dtype, device) -> torch.Tensor:
-    """Device scratch for one scan call of this shape (cached per device/size)."""
+def scan_workspace(B, T, H, Dh, dtype, device, stream=None) -> torch.Tensor:
+    """Device scratch for one scan call of this shape on ``stream`` (default:
+    the device's current stream).
+
+    A workspace may only be shared by calls ordered on one stream, so the
+    cache holds one per (device, stream, size): scans of the same shape on two
+    unordered streams get different workspaces."""
     lib = load_library()
     n = ctypes.c_size_t()
     _check("ratp_scan_workspace_bytes",
            lib.ratp_scan_workspace_bytes(B, T, H, Dh, _DTYPE[dtype], ctypes.byref(n)))
-    key = (str(device), n.value)
-    ws = _ws_cache.get(key)
-    if ws is None:
-        ws = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=device)   # zero before first use
-        _ws_cache[key] = ws
+    device = torch.device(device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    key = (str(device), stream.cuda_stream, n.value)
+    with _lock:
+        ws = _ws_cache.get(key)
+        if ws is None:
+            ws = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=device)   # zero before first use
+            if stream.cuda_stream != torch.cuda.current_stream(device).cuda_stream:
+                torch.cuda.current_stream(device).synchronize()   # the zero fill precedes its first use
+            _ws_cache[key] = ws
     return ws
 
 

@@ -12,7 +12,6 @@
 #include <string.h>
 
 #include <algorithm>
-#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -116,15 +115,6 @@ bool make_scan_map(CUtensorMap* m, const void* base, int B, int Tn, int C, int r
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Launch tags of the scan's self-validating chunk descriptors: unique per
-// launch within the process, never 0 (the value of a zero-filled workspace).
-std::atomic<unsigned int> g_scan_epoch{0};
-unsigned int next_scan_epoch() {
-  unsigned int e = ++g_scan_epoch;
-  while (e == 0) e = ++g_scan_epoch;
-  return e;
-}
-
 template <typename T, int NS, bool RESET>
 int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
                 int B, int Tn, int H, int Dh, int reset_L, const ScanGeom& geo,
@@ -136,7 +126,6 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   for (int s = 0; s < NS; ++s) p.h[s] = static_cast<T*>(h[s]);
   p.final_state = fs;
   p.ws = scan::carve(ws, geo.n_chunks, NS);
-  p.epoch = next_scan_epoch();
   p.B = B; p.Tn = Tn; p.C = H * Dh;
   p.reset_L = reset_L;
   p.l2_ahead = sm_count();   // about one ticket per SM ahead (measured: 100-200 alike)

@@ -19,7 +19,7 @@
 //     counter in launch order, so a CTA only waits on chunks whose CTAs have
 //     started.  Each lane of warp 0 owns two channels of the chunk's
 //     descriptor: it publishes its part of the aggregate map at once as
-//     epoch-tagged 64-bit words, then reads two predecessors per round trip
+//     tagged 64-bit words, then reads two predecessors per round trip
 //     and composes their aggregates until it meets an inclusive state.  x and
 //     g are read from HBM exactly once.
 //   * DRAM keeps streaming while CTAs compute: thread 0 of the CTA with ticket
@@ -60,18 +60,27 @@ struct Shape {
 };
 
 // Workspace layout (bytes), given n = total chunks and NS streams:
-//   [0, 256)                       ticket counter (u32) and abort word (u32 at
-//                                  byte 128), zeroed before each launch
+//   [0, 256)                       header: ticket counter (u32 at byte 0) and
+//                                  abort word (u32 at byte 128), zeroed before
+//                                  each launch; launch tag (u32 at byte 192),
+//                                  kept across launches
 //   agg  u64 [n][2(1+NS)][32]      aggregate map words, lane-minor
 //   incl u64 [n][2 NS][32]         inclusive-state words, lane-minor
 // Lane l of warp 0 owns channels 2l, 2l+1 of a chunk; word w of lane l holds
-// {epoch (high 32 bits), fp32 value (low 32 bits)}.  A 64-bit word is written
-// and read in one access, so a reader that sees the current launch's epoch
-// also sees its value: the descriptors need no flags, fences or reset, only
-// a zero fill before the workspace's first use (epoch 0 is never issued).
+// {tag (high 32 bits), fp32 value (low 32 bits)}.  A 64-bit word is written
+// and read in one access, so a reader that sees the current launch's tag also
+// sees its value: the descriptors need no flags, fences or reset, only a zero
+// fill before the workspace's first use (tag 0 is never issued).
+// The tag lives on the device: every CTA reads the stored tag before it draws
+// its ticket and uses the next one (1, 2, ..., 2^32 - 1, 1, ...); the CTA that
+// draws the last ticket stores it.  The ticket atomic is acq_rel, so every
+// other CTA's read of the stored tag happens before that store.  A launch
+// replayed from a CUDA graph therefore gets a fresh tag too, which a tag
+// fixed in the kernel parameters at capture time would not.
 struct Workspace {
   unsigned int* counter;
   unsigned int* abort;
+  unsigned int* tag;
   unsigned long long* agg;
   unsigned long long* incl;
 };
@@ -92,6 +101,7 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
   Workspace w;
   w.counter = reinterpret_cast<unsigned int*>(p);
   w.abort = reinterpret_cast<unsigned int*>(p + 128);
+  w.tag = reinterpret_cast<unsigned int*>(p + 192);
   p += 256;
   w.agg = reinterpret_cast<unsigned long long*>(p);
   p += align256(sizeof(unsigned long long) * n_chunks * 2 * (1 + NS) * kDescLanes);
@@ -99,8 +109,9 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
   return w;
 }
 
-// Bytes to zero before each launch: the ticket counter.
-inline size_t reset_bytes(long long) { return 256; }
+// Bytes to zero before each launch: the ticket counter and the abort word
+// (the launch tag at byte 192 is kept).
+inline size_t reset_bytes(long long) { return 192; }
 
 // L2 prefetch of one tile of a 3-D tensor map (no shared-memory destination).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
@@ -108,8 +119,8 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c
                :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2) : "memory");
 }
 
-__device__ __forceinline__ void put_word(unsigned long long* p, float v, unsigned int epoch) {
-  const unsigned long long w = ((unsigned long long)epoch << 32) | __float_as_uint(v);
+__device__ __forceinline__ void put_word(unsigned long long* p, float v, unsigned int tag) {
+  const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(w) : "memory");
 }
 
@@ -119,11 +130,25 @@ __device__ __forceinline__ unsigned long long get_word(const unsigned long long*
   return w;
 }
 
-__device__ __forceinline__ bool word_ok(unsigned long long w, unsigned int epoch) {
-  return (unsigned int)(w >> 32) == epoch;
+__device__ __forceinline__ bool word_ok(unsigned long long w, unsigned int tag) {
+  return (unsigned int)(w >> 32) == tag;
 }
+
 __device__ __forceinline__ float word_val(unsigned long long w) {
   return __uint_as_float((unsigned int)w);
+}
+
+// Draws this CTA's ticket and returns the launch tag (see Workspace).
+__device__ __forceinline__ unsigned int draw_ticket(const Workspace& ws, unsigned int n_tickets,
+                                                    unsigned int* ticket) {
+  unsigned int stored, t;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(stored) : "l"(ws.tag) : "memory");
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(ws.counter) : "memory");
+  const unsigned int tag = stored == 0xffffffffu ? 1u : stored + 1u;
+  if (t == n_tickets - 1u)
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" :: "l"(ws.tag), "r"(tag) : "memory");
+  *ticket = t;
+  return tag;
 }
 
 template <typename T, int NS>
@@ -131,7 +156,6 @@ struct Params {
   T* h[NS];
   float* final_state;     // nullable: [NS][B][C]
   Workspace ws;
-  unsigned int epoch;     // nonzero, unique per launch
   int B, Tn, C;           // Tn tokens, C = H * Dh channels per token
   int reset_L;            // chunk-local block length (RESET kernels only, >= 1)
   int l2_ahead;           // L2 prefetch distance in tickets (0: none)
@@ -164,7 +188,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   const T* s_g = reinterpret_cast<const T*>(smem);
   float* s_w = reinterpret_cast<float*>(smem + SM::kData);            // [NW][1 + NS][64]
   __shared__ __align__(8) uint64_t s_bar;
-  __shared__ unsigned int s_ticket;
+  __shared__ unsigned int s_ticket, s_tag;
   __shared__ float s_tot_a[kSlab];
   __shared__ float s_tot_b[NS][kSlab];
   __shared__ float s_carry[NS][kSlab];
@@ -178,12 +202,15 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
   };
   const uint32_t bar = sm100::smem_u32(&s_bar);
   if (tid == 0) {
-    s_ticket = atomicAdd(p.ws.counter, 1u);
+    unsigned int tk;
+    s_tag = draw_ticket(p.ws, (unsigned int)(p.n_chains * p.n_chunks_t), &tk);
+    s_ticket = tk;
     sm100::mbar_init(bar, 1);
     sm100::fence_barrier_init();
   }
   __syncthreads();
   const unsigned int ticket = s_ticket;
+  const unsigned int tag = s_tag;
   const int chunk = ticket / p.n_chains;     // chunk-major: predecessors started earlier
   const int chain = ticket % p.n_chains;
   const int b = chain / p.slabs;
@@ -245,7 +272,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
       if (tid < 32 && RATP_IN(desc, 1, (long long)p.n_chains * p.n_chunks_t)) {
 #pragma unroll
         for (int w = 0; w < 2 * NS; ++w)
-          put_word(p.ws.incl + (desc * 2 * NS + w) * kDescLanes + tid, 0.f, p.epoch);
+          put_word(p.ws.incl + (desc * 2 * NS + w) * kDescLanes + tid, 0.f, tag);
         if (tid == 0) {
           raise_error(RATP_ERR_TIMEOUT);
           atomicExch(p.ws.abort, 1u);
@@ -408,12 +435,12 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     [[maybe_unused]] const long long n_desc = (long long)p.n_chains * p.n_chunks_t;
     if (chunk > 0 && !drop && RATP_IN(desc, 1, n_desc)) {
       unsigned long long* dst = p.ws.agg + desc * WA * kDescLanes + lane;
-      put_word(dst + 0 * kDescLanes, s_tot_a[c0], p.epoch);
-      put_word(dst + 1 * kDescLanes, s_tot_a[c0 + 1], p.epoch);
+      put_word(dst + 0 * kDescLanes, s_tot_a[c0], tag);
+      put_word(dst + 1 * kDescLanes, s_tot_a[c0 + 1], tag);
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        put_word(dst + (2 + 2 * s) * kDescLanes, s_tot_b[s][c0], p.epoch);
-        put_word(dst + (3 + 2 * s) * kDescLanes, s_tot_b[s][c0 + 1], p.epoch);
+        put_word(dst + (2 + 2 * s) * kDescLanes, s_tot_b[s][c0], tag);
+        put_word(dst + (3 + 2 * s) * kDescLanes, s_tot_b[s][c0 + 1], tag);
       }
     }
     // a chunk whose first token restarts the recurrence needs no carry
@@ -441,9 +468,9 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
           inc[u] = true;
           ag[u] = true;
 #pragma unroll
-          for (int w = 0; w < WI; ++w) inc[u] = inc[u] && word_ok(wi[u][w], p.epoch);
+          for (int w = 0; w < WI; ++w) inc[u] = inc[u] && word_ok(wi[u][w], tag);
 #pragma unroll
-          for (int w = 0; w < WA; ++w) ag[u] = ag[u] && word_ok(wa[u][w], p.epoch);
+          for (int w = 0; w < WA; ++w) ag[u] = ag[u] && word_ok(wa[u][w], tag);
         }
         // how far this round gets: compose n aggregates, then maybe an inclusive
         int n = -1;
@@ -497,8 +524,8 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
       unsigned long long* dst = p.ws.incl + desc * (2 * NS) * kDescLanes + lane;
 #pragma unroll
       for (int s = 0; s < NS; ++s) {
-        put_word(dst + (2 * s) * kDescLanes, fmaf(s_tot_a[c0], cb0[s], s_tot_b[s][c0]), p.epoch);
-        put_word(dst + (2 * s + 1) * kDescLanes, fmaf(s_tot_a[c0 + 1], cb1[s], s_tot_b[s][c0 + 1]), p.epoch);
+        put_word(dst + (2 * s) * kDescLanes, fmaf(s_tot_a[c0], cb0[s], s_tot_b[s][c0]), tag);
+        put_word(dst + (2 * s + 1) * kDescLanes, fmaf(s_tot_a[c0 + 1], cb1[s], s_tot_b[s][c0 + 1]), tag);
       }
     }
 #pragma unroll

@@ -16,6 +16,7 @@ import recurrence_augmented_dilated_chunked_b200 as ratp
 from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
 from recurrence_augmented_dilated_chunked_b200._binding import RatpError
 from parity import assert_close, bits_equal, to64
+from cache_layout import LayoutShadow
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -118,8 +119,11 @@ def test_chunk_local_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, L):
     hk, hv = ratp.scan_prefill_kv(xk[:, :T].contiguous().to(DEV), xv[:, :T].contiguous().to(DEV),
                                   g[:, :T].contiguous().to(DEV), final_state=state, L=L)
     cache = ratp.KVCache(B, H, Dh, N, D, W, L=L)
+    shadow = LayoutShadow(cache, N)
     cache.pack(hk, hv)
     ratp.last_error()
+    shadow.prefill(hk, hv)
+    shadow.check("after pack")
 
     rk = oracle.scan(to64(xk[:, :T]), to64(g[:, :T]), L=L)
     rv = oracle.scan(to64(xv[:, :T]), to64(g[:, :T]), L=L)
@@ -131,6 +135,8 @@ def test_chunk_local_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, L):
         o = cache.decode_step(*[a.to(DEV) for a in args], state)
         ref = oc.decode_step(*[to64(a) for a in args])
         assert_close(o, ref, "bf16", "decode step %d (t=%d)" % (i, t))
+        shadow.append(state)
+        shadow.check("after decode step %d" % i)
     ratp.last_error()
     assert_close(state[0], oc.state[0], "f32", "final k state")
     assert_close(state[1], oc.state[1], "f32", "final v state")

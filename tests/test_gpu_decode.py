@@ -1,8 +1,9 @@
 """GPU parity of the D-compressed cache and the fused decode step.
 
-* layout: after the prefill hand-off and after every append, each dilated row
-  and ring row is bit-identical to the GPU's own recurrent key/value of the
-  position the layout rule assigns to it;
+* layout: after the prefill hand-off and after every decode step, the whole
+  dilated and ring regions of the GPU cache equal, bit for bit, the oracle's
+  pack of the GPU's own recurrent keys/values (the oracle's index map and
+  position rule; ``tests/cache_layout.py``);
 * numerics: decode outputs match the oracle's literal decode step (itself
   pinned to prefill attention) on the same seeded inputs;
 * the decode-from-32K-context and hybrid 7.6B-like workloads at full size,
@@ -17,14 +18,11 @@ import recurrence_augmented_dilated_chunked_b200 as ratp
 from recurrence_augmented_dilated_chunked_b200 import (WORKLOADS, decode_context, decode_inputs,
                                                        prefill_inputs)
 from recurrence_augmented_dilated_chunked_b200._binding import RatpError
-from parity import assert_close, bits_equal, to64
+from parity import assert_close, to64
+from cache_layout import LayoutShadow
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-
-
-def _dil(h, D, mask):
-    return 1 if (mask and mask[h]) else D
 
 
 @pytest.mark.parametrize("B,T,n,H,D,W,dense,Dh", [
@@ -44,22 +42,12 @@ def test_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, dense, Dh):
     hk, hv = ratp.scan_prefill_kv(xk[:, :T].contiguous().to(DEV), xv[:, :T].contiguous().to(DEV),
                                   g[:, :T].contiguous().to(DEV), final_state=state)
     cache = ratp.KVCache(B, H, Dh, N, D, W, head_mask=mask)
+    shadow = LayoutShadow(cache, N, mask)
     cache.pack(hk, hv)
     ratp.last_error()
-    # layout after pack: bit-identical to the GPU's own hk/hv rows
-    kc, vc = cache.dil_rows("k").cpu(), cache.dil_rows("v").cpu()
-    hk_c, hv_c = hk.cpu(), hv.cpu()
-    for h in range(H):
-        Dd = _dil(h, D, mask)
-        off, cap = cache.head_rows(h)
-        for s in range(T // Dd):
-            assert bits_equal(kc[:, off + s], hk_c[:, s * Dd + Dd - 1, h])
-            assert bits_equal(vc[:, off + s], hv_c[:, s * Dd + Dd - 1, h])
-    if W > 0:
-        kw = cache.ring("k").cpu()
-        for p in range(max(0, T - W), T):
-            assert bits_equal(kw[:, :, p % W], hk_c[:, p])
-    assert cache.lengths().cpu().tolist() == [T] * B
+    # layout after pack: the oracle's pack of the GPU's own hk/hv, bit for bit
+    shadow.prefill(hk, hv)
+    shadow.check("after pack")
 
     # oracle: fp64 scan of the same T tokens, pack, literal decode steps
     rk = oracle.scan(to64(xk[:, :T]), to64(g[:, :T]))
@@ -73,14 +61,9 @@ def test_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, dense, Dh):
         o = cache.decode_step(*[a.to(DEV) for a in args], state)
         ref = oc.decode_step(*[to64(a) for a in args])
         assert_close(o, ref, "bf16", "decode step %d" % i)
-        # appended rows are the bf16-rounded new state, bit for bit
-        st = state.cpu()
-        kc = cache.dil_rows("k")
-        for h in range(H):
-            Dd = _dil(h, D, mask)
-            if t % Dd == Dd - 1:
-                off, _ = cache.head_rows(h)
-                assert bits_equal(kc[:, off + t // Dd].cpu(), st[0, :, h].to(torch.bfloat16))
+        # appended rows are the bf16-rounded new state, where the oracle puts them
+        shadow.append(state)
+        shadow.check("after decode step %d" % i)
     ratp.last_error()
     assert cache.lengths().cpu().tolist() == [N] * B
     assert_close(state[0], oc.state[0], "f32", "final k state")

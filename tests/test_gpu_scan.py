@@ -100,3 +100,58 @@ def test_scan_empty_sequence_is_a_no_op(B, T):
     hk, hv = ratp.scan_prefill_kv(x, x, x)
     ratp.last_error()
     assert hk.shape == x.shape and hv.shape == x.shape
+
+
+def test_scan_graph_replays_with_new_inputs():
+    """A scan captured once in a CUDA graph and replayed with new inputs in
+    its static buffers matches the oracle on every replay: each replay's
+    chunk descriptors carry a fresh tag, so no look-back accepts a
+    predecessor's state from the previous replay."""
+    B, T, H, Dh = 2, 6000, 4, 128
+    x_in = [prefill_inputs(B, T, H, Dh, "bf16", gate_mean=1.0, gate_std=2.0, seed=40 + i)[1:]
+            for i in range(3)]
+    xk, xv, g = (t.to(DEV) for t in x_in[0])
+    hk, hv = torch.empty_like(xk), torch.empty_like(xv)
+    fs = torch.zeros(2, B, H, Dh, dtype=torch.float32, device=DEV)
+    ws = torch.zeros(ratp.scan_workspace(B, T, H, Dh, xk.dtype, DEV).numel(), dtype=torch.uint8,
+                     device=DEV)
+    ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, final_state=fs, workspace=ws)   # warm-up
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, final_state=fs, workspace=ws)
+    for i in (1, 2, 0, 1):
+        for dst, src in zip((xk, xv, g), x_in[i]):
+            dst.copy_(src)
+        graph.replay()
+        torch.cuda.synchronize()
+        ratp.last_error()
+        ref_k, ref_v = ratp.scan_prefill_kv(xk, xv, g)
+        assert bits_equal(hk, ref_k) and bits_equal(hv, ref_v), "replay with inputs %d" % i
+        rk = oracle.scan(to64(x_in[i][0]), to64(x_in[i][2]))
+        assert_close(hk, rk, "bf16", "replay with inputs %d" % i)
+        assert_close(fs[0], rk[:, -1], "f32", "final k state, replay with inputs %d" % i)
+    del graph
+
+
+def test_scan_on_two_unordered_streams():
+    """Scans of one shape issued on two streams with no order between them
+    use separate workspaces (the binding keeps one per stream) and both match
+    the oracle."""
+    B, T, H, Dh = 2, 8000, 8, 128
+    ins = [[t.to(DEV) for t in prefill_inputs(B, T, H, Dh, "bf16", seed=60 + i)[1:]] for i in range(2)]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = []
+    for _ in range(3):
+        for s, (xk, xv, g) in zip(streams, ins):
+            with torch.cuda.stream(s):
+                outs.append(ratp.scan_prefill_kv(xk, xv, g))
+    torch.cuda.synchronize()
+    ratp.last_error()
+    for i, (xk, xv, g) in enumerate(ins):
+        rk = oracle.scan(to64(xk), to64(g))
+        rv = oracle.scan(to64(xv), to64(g))
+        for hk, hv in outs[i::2]:
+            assert_close(hk, rk, "bf16", "stream %d hk" % i)
+            assert_close(hv, rv, "bf16", "stream %d hv" % i)

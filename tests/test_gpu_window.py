@@ -9,6 +9,7 @@ import recurrence_augmented_dilated_chunked_b200 as ratp
 from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
 from recurrence_augmented_dilated_chunked_b200._binding import RatpError
 from parity import assert_close, bits_equal, to64
+from cache_layout import LayoutShadow
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -105,12 +106,19 @@ def test_window_prefill_pack_decode_matches_oracle(B, T, n, H, D, W, L, dense):
     pre = [x[:, :T].contiguous().to(DEV) for x in (xk, xv, g)]
     hk, hv = ratp.scan_prefill_kv_window(*pre, L)
     cache = ratp.KVCache(B, H, Dh, N, D, W, head_mask=mask)
+    shadow = LayoutShadow(cache, N, mask)
     cache.attach_window(L)
     cache.pack(hk, hv)
     cache.pack_inputs(*pre)
+    shadow.prefill(hk, hv)
+    shadow.check("after pack")
     state = torch.zeros(2, B, H, Dh, dtype=torch.float32, device=DEV)
-    outs = [cache.decode_step(*[x[:, T + i].contiguous().to(DEV) for x in (q, xk, xv, g)], state)
-            for i in range(n)]
+    outs = []
+    for i in range(n):
+        outs.append(cache.decode_step(*[x[:, T + i].contiguous().to(DEV) for x in (q, xk, xv, g)],
+                                      state))
+        shadow.append(state)
+        shadow.check("after decode step %d" % i)
     ratp.last_error()
     rk = oracle.scan_window(to64(xk), to64(g), L)
     rv = oracle.scan_window(to64(xv), to64(g), L)
