@@ -122,11 +122,12 @@ int ratp_debug_guard_probe(void* stream);
  *   decode state.
  * workspace: device scratch of at least ratp_scan_workspace_bytes.  It must
  *   be zero-filled once before its first use; every call leaves it valid for
- *   the next one: each call zeroes its ticket counter on `stream` first, and
- *   its kernel tags the chunk descriptors with a fresh number kept in the
- *   workspace itself (so a call replayed from a CUDA graph gets a fresh tag
- *   as well; tags repeat after 2^32 - 1 calls on one workspace).  Calls
- *   sharing one workspace must be ordered on one stream.
+ *   the next one: each call clears its abort word on `stream` first, its
+ *   kernel returns the ticket counter to zero, and it tags the chunk
+ *   descriptors with a fresh number kept in the workspace itself (so a call
+ *   replayed from a CUDA graph gets a fresh tag as well; tags repeat after
+ *   2^32 - 1 calls on one workspace).  Calls sharing one workspace must be
+ *   ordered on one stream.
  *   h may alias x (in-place) only when T == 1.
  * Errors: ARG (null, B/T/H/Dh < 0), SHAPE (H*Dh not a multiple of 64), ALIGN,
  *   CAPACITY (workspace too small).  T == 0 or B == 0 is a no-op.

@@ -142,7 +142,7 @@ int launch_scan(const void* const* x, const void* g, void* const* h, float* fs,
   constexpr int smem = scan::Smem<T, NS>::kBytes;
   auto kernel = scan::scan_kernel<T, NS, scan::kRows, RESET>;
   if (!ensure_smem(kernel, smem)) return RATP_ERR_CUDA;
-  cudaError_t e = cudaMemsetAsync(ws, 0, scan::reset_bytes(geo.n_chunks), st);
+  cudaError_t e = cudaMemsetAsync(static_cast<char*>(ws) + scan::kResetOffset, 0, scan::kResetBytes, st);
   if (e != cudaSuccess) return RATP_ERR_CUDA;
   // one CTA per chunk; chunk tickets, not block indices, fix the order
   kernel<<<(unsigned)geo.n_chunks, scan::kThreads, smem, st>>>(tg, tx0, tx1, p);

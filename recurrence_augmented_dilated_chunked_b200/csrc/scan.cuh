@@ -60,10 +60,11 @@ struct Shape {
 };
 
 // Workspace layout (bytes), given n = total chunks and NS streams:
-//   [0, 256)                       header: ticket counter (u32 at byte 0) and
-//                                  abort word (u32 at byte 128), zeroed before
-//                                  each launch; launch tag (u32 at byte 192),
-//                                  kept across launches
+//   [0, 256)                       header: ticket word (u64 at byte 0: launch
+//                                  tag in the high 32 bits, ticket counter in
+//                                  the low 32), kept across launches; abort
+//                                  word (u32 at byte 128), zeroed before each
+//                                  launch
 //   agg  u64 [n][2(1+NS)][32]      aggregate map words, lane-minor
 //   incl u64 [n][2 NS][32]         inclusive-state words, lane-minor
 // Lane l of warp 0 owns channels 2l, 2l+1 of a chunk; word w of lane l holds
@@ -71,16 +72,17 @@ struct Shape {
 // and read in one access, so a reader that sees the current launch's tag also
 // sees its value: the descriptors need no flags, fences or reset, only a zero
 // fill before the workspace's first use (tag 0 is never issued).
-// The tag lives on the device: every CTA reads the stored tag before it draws
-// its ticket and uses the next one (1, 2, ..., 2^32 - 1, 1, ...); the CTA that
-// draws the last ticket stores it.  The ticket atomic is acq_rel, so every
-// other CTA's read of the stored tag happens before that store.  A launch
-// replayed from a CUDA graph therefore gets a fresh tag too, which a tag
-// fixed in the kernel parameters at capture time would not.
+// The tag lives on the device: every CTA draws its ticket with one 64-bit
+// atomic add on the ticket word, which also returns the tag stored there; the
+// launch uses the next tag (1, 2, ..., 2^32 - 1, 1, ...).  The CTA that draws
+// the last ticket stores {next tag, counter 0}; every other CTA's add comes
+// before that store in the word's order, so all of them saw the old tag, and
+// the next launch finds its counter at zero.  A launch replayed from a CUDA
+// graph therefore gets a fresh tag too, which a tag fixed in the kernel
+// parameters at capture time would not.
 struct Workspace {
-  unsigned int* counter;
+  unsigned long long* ticket;
   unsigned int* abort;
-  unsigned int* tag;
   unsigned long long* agg;
   unsigned long long* incl;
 };
@@ -99,9 +101,8 @@ inline size_t workspace_bytes(long long n_chunks, int NS) {
 inline Workspace carve(void* base, long long n_chunks, int NS) {
   char* p = static_cast<char*>(base);
   Workspace w;
-  w.counter = reinterpret_cast<unsigned int*>(p);
+  w.ticket = reinterpret_cast<unsigned long long*>(p);
   w.abort = reinterpret_cast<unsigned int*>(p + 128);
-  w.tag = reinterpret_cast<unsigned int*>(p + 192);
   p += 256;
   w.agg = reinterpret_cast<unsigned long long*>(p);
   p += align256(sizeof(unsigned long long) * n_chunks * 2 * (1 + NS) * kDescLanes);
@@ -109,9 +110,8 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
   return w;
 }
 
-// Bytes to zero before each launch: the ticket counter and the abort word
-// (the launch tag at byte 192 is kept).
-inline size_t reset_bytes(long long) { return 192; }
+// Zeroed before each launch: the abort word (the ticket word is kept).
+constexpr size_t kResetOffset = 128, kResetBytes = 64;
 
 // L2 prefetch of one tile of a 3-D tensor map (no shared-memory destination).
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
@@ -141,12 +141,13 @@ __device__ __forceinline__ float word_val(unsigned long long w) {
 // Draws this CTA's ticket and returns the launch tag (see Workspace).
 __device__ __forceinline__ unsigned int draw_ticket(const Workspace& ws, unsigned int n_tickets,
                                                     unsigned int* ticket) {
-  unsigned int stored, t;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(stored) : "l"(ws.tag) : "memory");
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(ws.counter) : "memory");
+  unsigned long long old;
+  asm volatile("atom.relaxed.gpu.global.add.u64 %0, [%1], 1;" : "=l"(old) : "l"(ws.ticket) : "memory");
+  const unsigned int t = (unsigned int)old, stored = (unsigned int)(old >> 32);
   const unsigned int tag = stored == 0xffffffffu ? 1u : stored + 1u;
   if (t == n_tickets - 1u)
-    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" :: "l"(ws.tag), "r"(tag) : "memory");
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(ws.ticket), "l"((unsigned long long)tag << 32)
+                 : "memory");
   *ticket = t;
   return tag;
 }
