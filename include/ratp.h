@@ -83,13 +83,16 @@ int ratp_device_sm_count(int* sms);
  *                            no descriptor, so its successor's wait runs out;
  *   RATP_FAULT_ATTN_DROP_K   the first CTA of the tensor-core attention never
  *                            loads its K tile number `arg`, so the MMA's wait
- *                            runs out.
+ *                            runs out;
+ *   RATP_FAULT_FUSED_DROP_UNIT  the fused prefill never raises the done flag
+ *                            of recurrence unit `arg` (unit = (b*H + h) *
+ *                            ceil(T/256) + t/256), so the waits on it run out.
  * A wait that runs out ends its kernel early with RATP_ERR_TIMEOUT in the
  * device error word (outputs are then undefined); the context stays usable.
  * Returns RATP_ERR_ARG for an unknown kind, RATP_ERR_CUDA if the device
  * update fails.  Not thread-safe with concurrent launches. */
 enum { RATP_FAULT_NONE = 0, RATP_FAULT_SPIN_LIMIT = 1, RATP_FAULT_SCAN_DROP = 2,
-       RATP_FAULT_ATTN_DROP_K = 3 };
+       RATP_FAULT_ATTN_DROP_K = 3, RATP_FAULT_FUSED_DROP_UNIT = 4 };
 int ratp_debug_fault(int kind, long long arg);
 
 /* ------------------------------------------------------------------------
@@ -241,6 +244,40 @@ int ratp_dilated_attn_prefill(const void* q, const void* hk, const void* hv, voi
 int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv, void* o,
                                    int B, int T, int H, int Dh, int D, int W,
                                    const uint8_t* head_mask, int dtype, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Fused prefill: the recurrence of both streams and the dilated (+ windowed,
+ * head-wise hybrid) attention over it in one launch (the full-sequence
+ * recurrence of the write-up's section 2.1 feeding the dilated attention of
+ * its section 1 and of the RAT+ abstract).
+ *
+ * Computes what ratp_scan_prefill_kv followed by ratp_dilated_attn_prefill
+ * computes: hk = scan(xk, g), hv = scan(xv, g), final_state = the fp32 state
+ * at position T-1 ([2][B][H][Dh], k then v; nullable), and o = attention of q
+ * over hk, hv with dilation D, window W and head_mask (HOST array of H bytes,
+ * nonzero = dense head; or NULL).  Inside the launch, scan warps compute the
+ * recurrence 256 positions of one (b, h) at a time, ahead of the tensor-core
+ * pipeline, which waits (bounded) on a per-unit flag before it loads keys a
+ * unit holds; the recurrence runs in a different association order than
+ * ratp_scan_prefill_kv, so results agree to rounding, not bit for bit.
+ * q, xk, xv, g, hk, hv, o: [B][T][H][Dh] bf16, Dh = 128, device, 16-byte
+ * aligned; hk and hv are written (they are outputs, and the attention reads
+ * its keys back from them, mostly out of L2).
+ * workspace: device scratch of ratp_prefill_fused_workspace_bytes bytes,
+ *   zero-filled once before its first use; like the scan workspace it tags
+ *   its descriptors and flags with a fresh number per call, kept in the
+ *   workspace itself, and calls sharing one workspace must be ordered on one
+ *   stream.
+ * Errors: ARG, SHAPE, ALIGN, CAPACITY (workspace too small), UNSUPPORTED
+ *   (not bf16 or Dh != 128).  B, T or H == 0 is a no-op.  A bounded wait that
+ *   ran out sets RATP_ERR_TIMEOUT in the device error word (outputs are then
+ *   undefined).
+ * ---------------------------------------------------------------------- */
+int ratp_prefill_fused_workspace_bytes(int B, int T, int H, int Dh, size_t* bytes);
+int ratp_prefill_fused(const void* q, const void* xk, const void* xv, const void* g,
+                       void* hk, void* hv, void* o, float* final_state,
+                       int B, int T, int H, int Dh, int D, int W, const uint8_t* head_mask, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
  * Per-sample dilation in one launch (the batch composition of the write-up's

@@ -19,6 +19,8 @@ from ._binding import (  # noqa: F401
     guard_line,
     last_error,
     load_library,
+    prefill_fused,
+    prefill_fused_workspace,
     scan_prefill,
     scan_prefill_kv,
     scan_prefill_kv_noalloc,

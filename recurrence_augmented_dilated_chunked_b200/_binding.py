@@ -77,6 +77,8 @@ _SIGS = {
     "ratp_dilated_attn_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_simt": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_per_sample": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I, _P], _I),
+    "ratp_prefill_fused_workspace_bytes": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
+    "ratp_prefill_fused": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _SZ, _P], _I),
     "ratp_cache_bytes": ([_I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)], _I),
     "ratp_cache_init": ([ctypes.POINTER(CacheStruct), _P, _SZ, _I, _I, _I, _I, _I, _I, _P, _P], _I),
     "ratp_cache_pack": ([ctypes.POINTER(CacheStruct), _P, _P, _I, _P], _I),
@@ -312,6 +314,59 @@ def dilated_attn_prefill_per_sample(q, hk, hv, D_per_sample, W=0, head_mask=None
     return out
 
 
+_fused_ws_cache = {}
+
+
+def prefill_fused_workspace(B, T, H, Dh, device, stream=None) -> torch.Tensor:
+    """Device scratch for one fused prefill of this shape on ``stream`` (default:
+    the device's current stream), cached per (device, stream, size) like the
+    scan workspace."""
+    lib = load_library()
+    n = ctypes.c_size_t()
+    _check("ratp_prefill_fused_workspace_bytes",
+           lib.ratp_prefill_fused_workspace_bytes(B, T, H, Dh, ctypes.byref(n)))
+    device = torch.device(device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    key = (str(device), stream.cuda_stream, n.value)
+    with _lock:
+        ws = _fused_ws_cache.get(key)
+        if ws is None:
+            ws = torch.zeros(max(n.value, 256), dtype=torch.uint8, device=device)   # zero before first use
+            if stream.cuda_stream != torch.cuda.current_stream(device).cuda_stream:
+                torch.cuda.current_stream(device).synchronize()
+            _fused_ws_cache[key] = ws
+    return ws
+
+
+def prefill_fused(q, xk, xv, g, D, W=0, head_mask=None, hk=None, hv=None, out=None, final_state=None,
+                  workspace=None):
+    """(o, hk, hv): the key/value recurrence and the dilated (+ windowed)
+    attention over it in one launch; bf16, head dim 128."""
+    lib = load_library()
+    _need(q, "q")
+    for t, nm in ((xk, "xk"), (xv, "xv"), (g, "g")):
+        _need(t, nm, q.dtype)
+    B, T, H, Dh = q.shape
+    if xk.shape != q.shape or xv.shape != q.shape or g.shape != q.shape:
+        raise ValueError("q, xk, xv, g must have one shape")
+    hk = torch.empty_like(xk) if hk is None else hk
+    hv = torch.empty_like(xv) if hv is None else hv
+    out = torch.empty_like(q) if out is None else out
+    for t, nm in ((hk, "hk"), (hv, "hv"), (out, "out")):
+        _need(t, nm, q.dtype)
+    if final_state is not None:
+        _need(final_state, "final_state", torch.float32)
+    if q.dtype not in _DTYPE:
+        raise ValueError("unsupported dtype %s" % q.dtype)
+    ws = workspace if workspace is not None else prefill_fused_workspace(B, T, H, Dh, q.device)
+    _buf, mp = _mask_buf(head_mask, H)
+    _check("ratp_prefill_fused", lib.ratp_prefill_fused(
+        _ptr(q), _ptr(xk), _ptr(xv), _ptr(g), _ptr(hk), _ptr(hv), _ptr(out), _ptr(final_state),
+        B, T, H, Dh, int(D), int(W), mp, _DTYPE[q.dtype], _ptr(ws), ws.numel(), _stream(q)))
+    return out, hk, hv
+
+
 def last_error(device=None):
     """Synchronise and raise if any kernel recorded a device-side error."""
     lib = load_library()
@@ -320,7 +375,7 @@ def last_error(device=None):
     _check("ratp_last_error", lib.ratp_last_error(s))
 
 
-FAULT_NONE, FAULT_SPIN_LIMIT, FAULT_SCAN_DROP, FAULT_ATTN_DROP_K = 0, 1, 2, 3
+FAULT_NONE, FAULT_SPIN_LIMIT, FAULT_SCAN_DROP, FAULT_ATTN_DROP_K, FAULT_FUSED_DROP_UNIT = 0, 1, 2, 3, 4
 
 
 def debug_fault(kind: int, arg: int = 0):

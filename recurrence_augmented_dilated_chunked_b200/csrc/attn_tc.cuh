@@ -58,6 +58,7 @@
 // is released.
 #pragma once
 #include "sm100.cuh"
+#include "fused.cuh"
 
 namespace ratp {
 namespace attn_tc {
@@ -70,6 +71,11 @@ constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 192;
+// The fused prefill (recurrence and attention in one launch) adds two scan
+// warps per CTA (warps 6-7, fused.cuh) and their scratch.
+constexpr int kScanWarp0 = 6;
+constexpr int kThreadsFused = 256;
+constexpr uint32_t kScanScratch = 20 * 32 * 4;
 constexpr uint32_t kQHalf = BM * 64 * 2;       // Q: 128 rows x 64 columns: 16 KB
 constexpr uint32_t kQTile = 2 * kQHalf;        // 32 KB
 constexpr uint32_t kKHalf = BN * 64 * 2;       // K/V: 64 rows x 64 columns: 8 KB
@@ -80,7 +86,9 @@ constexpr uint32_t kOffV = kOffK + 2 * kKTile; // 2 stages
 constexpr uint32_t kOffBar = kOffV + 2 * kKTile;
 // barriers: qfull qempty kfull[2] kempty[2] vfull[2] sfull sfree pfull[2] pvdone[2] final
 constexpr uint32_t kNumBars = 15;
-constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + TMEM slot, abort, alignment
+constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + TMEM slot, abort, tag, alignment
+constexpr uint32_t kOffScan = kOffBar + kNumBars * 8 + 16;               // fused: scan scratch
+constexpr uint32_t kSmemBytesFused = kSmemBytes + kScanScratch;
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0;      // S: 64 columns
 constexpr uint32_t kColP = 64;     // P buffer b at 64 + 32 b
@@ -90,7 +98,7 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units
 // loops stay rolled, which keeps the softmax loop's code compact (measured
 // 2% faster than unrolling them).
 constexpr int kColdUnroll = 1;
-static_assert(kCtasPerSm * (kSmemBytes + 1024) <= 233472, "two CTAs per SM");
+static_assert(kCtasPerSm * (kSmemBytesFused + 1024) <= 233472, "two CTAs per SM");
 
 constexpr int kMaxDil = 4;                 // distinct dilations D > 1 in one launch
 constexpr int kMaxSeg = 2 + kMaxDil;
@@ -125,6 +133,17 @@ struct Params {
   uint8_t dense_list[RATP_MAX_HEADS];
   uint8_t dil_list[RATP_MAX_HEADS];
   uint16_t samples[kMaxSamples];   // samples grouped by dilation (per-sample mode)
+  // fused prefill: items in ascending order (query tile major, then b, h),
+  // head h dense where bit h of dense_bits is set, else dilation dil_D[0]
+  unsigned long long dense_bits[RATP_MAX_HEADS / 64];
+  fused::ScanParams scan;
+  int tag_ctas;                    // CTAs of the launch (each draws the launch tag once)
+};
+
+// The fused prefill's inputs x_k, x_v, g as [B][T][H][128] views (the L2
+// prefetch of the scan's next unit).
+struct ScanMaps {
+  CUtensorMap xk, xv, g;
 };
 
 struct Item {
@@ -132,22 +151,36 @@ struct Item {
   bool dense;
 };
 
+template <bool FUSED>
 __device__ __forceinline__ Item make_item(const Params& p, int idx) {
-  int s = 0;
-  while (s + 1 < p.n_seg && idx >= p.seg[s + 1].begin) ++s;
-  const Segment& g = p.seg[s];
   Item it;
-  idx -= g.begin;
-  const int per = g.n_b * g.n_h;
-  const int qi = idx / per;
-  const int rem = idx - qi * per;
-  const int bi = rem / g.n_h;
-  const int hi = rem - bi * g.n_h;
-  it.b = g.b_off < 0 ? bi : (int)p.samples[g.b_off + bi];
-  it.h = g.heads == kHeadsDense ? (int)p.dense_list[hi] : g.heads == kHeadsDil ? (int)p.dil_list[hi] : hi;
-  it.cls = g.cls < 0 ? 0 : g.cls;
-  it.dense = g.cls < 0;
-  it.t0 = (p.NQ - 1 - qi) * BM;
+  if (FUSED) {
+    // ascending: every unit an item reads is scanned by an item that comes
+    // no later in this order
+    const int per = p.B * p.H;
+    const int qi = idx / per;
+    const int rem = idx - qi * per;
+    it.b = rem / p.H;
+    it.h = rem - it.b * p.H;
+    it.cls = 0;
+    it.dense = ((p.dense_bits[it.h >> 6] >> (it.h & 63)) & 1ull) != 0ull || p.dil_D[0] == 1;
+    it.t0 = qi * BM;
+  } else {
+    int s = 0;
+    while (s + 1 < p.n_seg && idx >= p.seg[s + 1].begin) ++s;
+    const Segment& g = p.seg[s];
+    idx -= g.begin;
+    const int per = g.n_b * g.n_h;
+    const int qi = idx / per;
+    const int rem = idx - qi * per;
+    const int bi = rem / g.n_h;
+    const int hi = rem - bi * g.n_h;
+    it.b = g.b_off < 0 ? bi : (int)p.samples[g.b_off + bi];
+    it.h = g.heads == kHeadsDense ? (int)p.dense_list[hi] : g.heads == kHeadsDil ? (int)p.dil_list[hi] : hi;
+    it.cls = g.cls < 0 ? 0 : g.cls;
+    it.dense = g.cls < 0;
+    it.t0 = (p.NQ - 1 - qi) * BM;
+  }
   it.t_last = min(it.t0 + BM - 1, p.T - 1);
   if (it.dense) {
     it.Dd = 1;
@@ -165,11 +198,52 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
 }
 
 
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+// Waits (whole warp) until every unit an item reads is scanned: the units
+// 0 .. (item's own) of its (b, h).  Then the TMA loads that lane 0 issues
+// next see the scan's stores.  False if the wait ran out or another CTA
+// aborted.
+__device__ __forceinline__ bool wait_units(const Params& p, const Item& it, unsigned int tag, int lane,
+                                           volatile int* s_abort) {
+  const long long first = ((long long)it.b * p.H + it.h) * p.NQ;
+  const int last = it.t0 / BM;
+  const unsigned long long t0 = global_ns();
+  unsigned int polls = 0;
+  for (int j0 = 0; j0 <= last; j0 += 32) {
+    const int j = j0 + lane;
+    bool done = j > last;
+    while (true) {
+      if (!done && RATP_IN(first + j, 1, (long long)p.B * p.H * p.NQ))
+        done = fused::ld_acquire(p.scan.ws.flags + first + j) == tag;
+      if (__all_sync(0xffffffffu, done)) break;
+      bool give_up = false;
+      if ((++polls & 15u) == 0u)
+        give_up = *s_abort || fused::aborted(p.scan.ws) || global_ns() - t0 > spin_timeout();
+      if (__any_sync(0xffffffffu, give_up)) {
+        if (lane == 0) {
+          *s_abort = 1;
+          fused::abort_all(p.scan.ws);
+        }
+        return false;
+      }
+      __nanosleep(32);
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    fused::fence_proxy_async_global();
+  }
+  __syncwarp();
+  return true;
+}
+
+template <bool FUSED>
+__global__ void __launch_bounds__(FUSED ? kThreadsFused : kThreads, kCtasPerSm)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             const __grid_constant__ CUtensorMap tm_kpos,
             const __grid_constant__ CUtensorMap tm_vpos,
             const __grid_constant__ DilMaps tm_dil,
+            const __grid_constant__ ScanMaps tm_scan,
             const __grid_constant__ Params p) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -190,6 +264,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t b_final = bar0 + 14 * 8;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 4);
+  unsigned int* s_tag = reinterpret_cast<unsigned int*>(smem + kOffBar + kNumBars * 8 + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -208,6 +283,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     }
     mbar_init(b_final, 1);
     *s_abort = 0;
+    if (FUSED) *s_tag = fused::draw_tag(p.scan.ws, (unsigned int)p.tag_ctas);
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -227,20 +303,22 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
+  const unsigned int tag = FUSED ? *s_tag : 0u;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     // Tile n (stage n%2): K once S = Q K^T of tile n-2 read the stage; at an
     // item's first tile then Q, once the previous item's last S = Q K^T is
     // done (its K load is already under way); V once O += P V of tile n-2
-    // read the stage.  The next item's Q is prefetched into L2 one item
-    // ahead, so its load at the item boundary is an L2 hit.
-    if (lane == 0) {
-      int n = 0, li = 0, nq = 0;
-      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};   // last tile loaded per stage
-      bool ok = true;
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
-        const Item it = make_item(p, idx);
+    // read the stage.  The fused prefill first waits (whole warp) for the
+    // recurrence units the item reads.
+    int n = 0, li = 0, nq = 0;
+    int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};   // last tile loaded per stage
+    bool ok = true;
+    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
+      const Item it = make_item<FUSED>(p, idx);
+      if (FUSED && !wait_units(p, it, tag, lane, s_abort)) ok = false;
+      if (ok && lane == 0) {
         for (int j = 0; j < it.n_tiles; ++j, ++n) {
           const int st = n & 1;
           const bool pos = (j < it.n_win) || it.dense;
@@ -270,8 +348,11 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           last_v[st] = n;
         }
       }
-      // let the copies in flight land before the CTA ends (after an abort
-      // they may never have been consumed)
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+    }
+    // let the copies in flight land before the CTA ends (after an abort
+    // they may never have been consumed)
+    if (lane == 0) {
       if (nq > 0) mbar_drain(b_qfull, (nq - 1) & 1);
       for (int st = 0; st < 2; ++st) {
         if (last_k[st] >= 0) mbar_drain(b_kfull + 8 * st, (last_k[st] >> 1) & 1);
@@ -324,7 +405,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         return true;
       };
       for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
-        const int n_tiles = make_item(p, idx).n_tiles;
+        const int n_tiles = make_item<FUSED>(p, idx).n_tiles;
         if (!mbar_wait(b_qfull, li & 1, s_abort)) { ok = false; break; }
         if (!issue_s(n)) { ok = false; break; }
         for (int j = 1; j < n_tiles; ++j) {
@@ -340,7 +421,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_drain(b_final, 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp < kSoftmaxWarps) {
     // ------------------------------------------------------------ softmax
     const int r = warp * 32 + lane;                  // query row within the tile (TMEM lane)
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
@@ -352,7 +433,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     int n = 0;                                       // tiles so far
     bool ok = true;
     for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
-      const Item it = make_item(p, idx);
+      const Item it = make_item<FUSED>(p, idx);
       const int t = it.t0 + r;
       const int lim_dil = it.dense ? (t + 1) : (max(0, t - p.W_eff + 1) / it.Dd);
       const int w_lo = max(t - p.W_eff + 1, 0);
@@ -497,6 +578,30 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       tc_fence_before();
+    }
+  }
+
+  if (FUSED && warp >= kScanWarp0) {
+    // ------------------------------------------------------------ scan (fused prefill)
+    // This CTA's items in its own order, each item's unit scanned ahead of
+    // its attention; lane 0 of the first scan warp prefetches the next unit's
+    // inputs into L2.
+    const int sw = warp - kScanWarp0;
+    float* s_map = reinterpret_cast<float*>(smem + kOffScan);
+    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
+      const Item it = make_item<FUSED>(p, idx);
+      if (sw == 0 && lane == 0 && idx + (int)gridDim.x < p.n_items) {
+        const Item nx = make_item<FUSED>(p, idx + gridDim.x);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tma_prefetch_l2_4d(&tm_scan.g, 64 * c, nx.h, nx.t0, nx.b);
+          tma_prefetch_l2_4d(&tm_scan.xk, 64 * c, nx.h, nx.t0, nx.b);
+          tma_prefetch_l2_4d(&tm_scan.xv, 64 * c, nx.h, nx.t0, nx.b);
+        }
+      }
+      // a unit whose wait ran out still publishes (a zero carry), so that no
+      // other CTA waits on it; the error word holds the timeout
+      fused::scan_unit(p.scan, p.B, p.T, p.H, it.b, it.h, it.t0 / BM, sw, lane, tag, s_map, 1);
     }
   }
 

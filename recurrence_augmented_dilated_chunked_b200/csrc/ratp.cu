@@ -380,10 +380,71 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
       dm.v[c] = tvp;
     }
   }
-  if (!ensure_smem(attn_tc::attn_kernel, (int)attn_tc::kSmemBytes)) return RATP_ERR_CUDA;
+  attn_tc::ScanMaps sm_unused;
+  memset(&sm_unused, 0, sizeof(sm_unused));
+  auto kernel = attn_tc::attn_kernel<false>;
+  if (!ensure_smem(kernel, (int)attn_tc::kSmemBytes)) return RATP_ERR_CUDA;
   const int slots = attn_tc::kCtasPerSm * sm_count();
   const int grid = p.n_items < slots ? p.n_items : slots;
-  attn_tc::attn_kernel<<<grid, attn_tc::kThreads, attn_tc::kSmemBytes, st>>>(tq, tkp, tvp, dm, p);
+  kernel<<<grid, attn_tc::kThreads, attn_tc::kSmemBytes, st>>>(tq, tkp, tvp, dm, sm_unused, p);
+  return launch_status();
+}
+
+// Fused prefill: the recurrence of both streams and the attention in one
+// launch (attn_kernel<true>: scan warps ahead of the tensor-core pipeline).
+int launch_prefill_fused(const void* q, const void* xk, const void* xv, const void* g, void* hk, void* hv,
+                         void* o, float* fs, int B, int T, int H, int D, int W, const uint8_t* head_mask,
+                         void* ws, size_t ws_bytes, cudaStream_t st) {
+  attn_tc::Params p;
+  memset(&p, 0, sizeof(p));
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.B = B; p.T = T; p.H = H; p.W_eff = W > 0 ? W : 1;
+  p.NQ = (T + attn_tc::BM - 1) / attn_tc::BM;
+  const long long n_units = (long long)B * H * p.NQ;
+  if (n_units > 0x7fffffffll) return RATP_ERR_SHAPE;
+  if (ws_bytes < fused::workspace_bytes(n_units)) return RATP_ERR_CAPACITY;
+  int rc = read_mask(head_mask, H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
+  if (rc) return rc;
+  p.n_items = (int)n_units;
+  p.n_cls = D > 1 ? 1 : 0;
+  p.dil_D[0] = D;
+  p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
+  p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
+  p.scan.xk = static_cast<const __nv_bfloat16*>(xk);
+  p.scan.xv = static_cast<const __nv_bfloat16*>(xv);
+  p.scan.g = static_cast<const __nv_bfloat16*>(g);
+  p.scan.hk = static_cast<__nv_bfloat16*>(hk);
+  p.scan.hv = static_cast<__nv_bfloat16*>(hv);
+  p.scan.final_state = fs;
+  p.scan.ws = fused::carve(ws, n_units);
+  p.scan.NQ = p.NQ;
+  const long long row = (long long)H * 128, bat = (long long)T * row;
+  constexpr int qr = attn_tc::BM, kr = attn_tc::BN;
+  CUtensorMap tq, tkp, tvp;
+  attn_tc::DilMaps dm;
+  attn_tc::ScanMaps sm;
+  memset(&dm, 0, sizeof(dm));
+  if (!make_map(&tq, q, 0, B, T, H, row, bat, qr) || !make_map(&tkp, hk, 0, B, T, H, row, bat, kr) ||
+      !make_map(&tvp, hv, 0, B, T, H, row, bat, kr) || !make_map(&sm.xk, xk, 0, B, T, H, row, bat, qr) ||
+      !make_map(&sm.xv, xv, 0, B, T, H, row, bat, qr) || !make_map(&sm.g, g, 0, B, T, H, row, bat, qr))
+    return RATP_ERR_CUDA;
+  const long long n_slots = D > 1 ? T / D : 0;
+  if (n_slots >= 1) {
+    if (!make_map(&dm.k[0], hk, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat, kr) ||
+        !make_map(&dm.v[0], hv, (long long)(D - 1) * row, B, n_slots, H, (long long)D * row, bat, kr))
+      return RATP_ERR_CUDA;
+  } else {
+    dm.k[0] = tkp;   // no dilated slot exists for any query: never read
+    dm.v[0] = tvp;
+  }
+  auto kernel = attn_tc::attn_kernel<true>;
+  if (!ensure_smem(kernel, (int)attn_tc::kSmemBytesFused)) return RATP_ERR_CUDA;
+  const int slots = attn_tc::kCtasPerSm * sm_count();
+  const int grid = p.n_items < slots ? p.n_items : slots;
+  p.tag_ctas = grid;
+  if (cudaMemsetAsync(static_cast<char*>(ws) + fused::kResetOffset, 0, fused::kResetBytes, st) != cudaSuccess)
+    return RATP_ERR_CUDA;
+  kernel<<<grid, attn_tc::kThreadsFused, attn_tc::kSmemBytesFused, st>>>(tq, tkp, tvp, dm, sm, p);
   return launch_status();
 }
 
@@ -523,31 +584,34 @@ int ratp_debug_guard_probe(void* stream) {
 }
 
 int ratp_debug_fault(int kind, long long arg) {
-  unsigned long long timeout = ratp::kSpinTimeoutNs;
-  long long scan = -1, attn = -1;
+  // each kind sets one device variable; RATP_FAULT_NONE restores all four
+  const long long none = -1;
+  const unsigned long long timeout =
+      (kind == RATP_FAULT_SPIN_LIMIT && arg > 0) ? (unsigned long long)arg : ratp::kSpinTimeoutNs;
+  bool ok = true;
   switch (kind) {
-    case RATP_FAULT_NONE: break;
-    case RATP_FAULT_SPIN_LIMIT: if (arg > 0) timeout = (unsigned long long)arg; break;
-    case RATP_FAULT_SCAN_DROP: scan = arg; break;
-    case RATP_FAULT_ATTN_DROP_K: attn = arg; break;
-    default: return RATP_ERR_ARG;
+    case RATP_FAULT_NONE:
+      ok = cudaMemcpyToSymbol(ratp::g_spin_timeout_ns, &timeout, sizeof(timeout)) == cudaSuccess &&
+           cudaMemcpyToSymbol(ratp::g_fault_scan_ticket, &none, sizeof(none)) == cudaSuccess &&
+           cudaMemcpyToSymbol(ratp::g_fault_attn_ktile, &none, sizeof(none)) == cudaSuccess &&
+           cudaMemcpyToSymbol(ratp::g_fault_fused_unit, &none, sizeof(none)) == cudaSuccess;
+      break;
+    case RATP_FAULT_SPIN_LIMIT:
+      ok = cudaMemcpyToSymbol(ratp::g_spin_timeout_ns, &timeout, sizeof(timeout)) == cudaSuccess;
+      break;
+    case RATP_FAULT_SCAN_DROP:
+      ok = cudaMemcpyToSymbol(ratp::g_fault_scan_ticket, &arg, sizeof(arg)) == cudaSuccess;
+      break;
+    case RATP_FAULT_ATTN_DROP_K:
+      ok = cudaMemcpyToSymbol(ratp::g_fault_attn_ktile, &arg, sizeof(arg)) == cudaSuccess;
+      break;
+    case RATP_FAULT_FUSED_DROP_UNIT:
+      ok = cudaMemcpyToSymbol(ratp::g_fault_fused_unit, &arg, sizeof(arg)) == cudaSuccess;
+      break;
+    default:
+      return RATP_ERR_ARG;
   }
-  // a drop keeps the current wait bound; a new bound keeps the drops
-  if (kind == RATP_FAULT_SCAN_DROP || kind == RATP_FAULT_ATTN_DROP_K) {
-    if (cudaMemcpyFromSymbol(&timeout, ratp::g_spin_timeout_ns, sizeof(timeout)) != cudaSuccess) return RATP_ERR_CUDA;
-    long long other = -1;
-    if (cudaMemcpyFromSymbol(&other, kind == RATP_FAULT_SCAN_DROP ? ratp::g_fault_attn_ktile : ratp::g_fault_scan_ticket,
-                             sizeof(other)) != cudaSuccess) return RATP_ERR_CUDA;
-    if (kind == RATP_FAULT_SCAN_DROP) attn = other; else scan = other;
-  } else if (kind == RATP_FAULT_SPIN_LIMIT) {
-    if (cudaMemcpyFromSymbol(&scan, ratp::g_fault_scan_ticket, sizeof(scan)) != cudaSuccess ||
-        cudaMemcpyFromSymbol(&attn, ratp::g_fault_attn_ktile, sizeof(attn)) != cudaSuccess) return RATP_ERR_CUDA;
-  }
-  if (cudaMemcpyToSymbol(ratp::g_spin_timeout_ns, &timeout, sizeof(timeout)) != cudaSuccess ||
-      cudaMemcpyToSymbol(ratp::g_fault_scan_ticket, &scan, sizeof(scan)) != cudaSuccess ||
-      cudaMemcpyToSymbol(ratp::g_fault_attn_ktile, &attn, sizeof(attn)) != cudaSuccess)
-    return RATP_ERR_CUDA;
-  return RATP_OK;
+  return ok ? RATP_OK : RATP_ERR_CUDA;
 }
 
 int ratp_device_sm_count(int* sms) {
@@ -664,6 +728,30 @@ int ratp_dilated_attn_prefill(const void* q, const void* hk, const void* hv, voi
   if (dtype == RATP_BF16 && Dh == 128)
     return launch_attn_tc(q, hk, hv, o, B, T, H, nullptr, D, W, head_mask, st);
   return launch_attn_simt(q, hk, hv, o, B, T, H, Dh, D, W, head_mask, dtype, st);
+}
+
+int ratp_prefill_fused_workspace_bytes(int B, int T, int H, int Dh, size_t* bytes) {
+  if (!bytes || B < 0 || T < 0 || H < 0) return RATP_ERR_ARG;
+  if (Dh != 128) return RATP_ERR_UNSUPPORTED;
+  const long long n_units = (long long)B * H * ((T + attn_tc::BM - 1) / attn_tc::BM);
+  if (n_units > 0x7fffffffll) return RATP_ERR_SHAPE;
+  *bytes = fused::workspace_bytes(n_units);
+  return RATP_OK;
+}
+
+int ratp_prefill_fused(const void* q, const void* xk, const void* xv, const void* g,
+                       void* hk, void* hv, void* o, float* final_state,
+                       int B, int T, int H, int Dh, int D, int W, const uint8_t* head_mask, int dtype,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_attn_args(q, hk, hv, o, B, T, H, Dh, D, W, dtype);
+  if (rc) return rc;
+  if (dtype != RATP_BF16 || Dh != 128) return RATP_ERR_UNSUPPORTED;
+  if ((long long)B * T * H == 0) return RATP_OK;
+  if (!xk || !xv || !g || !workspace) return RATP_ERR_ARG;
+  if (!aligned16(xk) || !aligned16(xv) || !aligned16(g) || !aligned16(workspace)) return RATP_ERR_ALIGN;
+  if (final_state != nullptr && !aligned16(final_state)) return RATP_ERR_ALIGN;
+  return launch_prefill_fused(q, xk, xv, g, hk, hv, o, final_state, B, T, H, D, W, head_mask, workspace,
+                              workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int ratp_dilated_attn_prefill_per_sample(const void* q, const void* hk, const void* hv, void* o,
