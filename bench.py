@@ -167,7 +167,7 @@ class ClockSampler:
 
 KERNEL_SOURCES = {
     "scan_kv": ["scan.cuh", "common.cuh", "sm100.cuh"],
-    "dilated_attn": ["attn_tc.cuh", "common.cuh", "sm100.cuh"],
+    "dilated_attn": ["attn_tc.cuh", "fused.cuh", "common.cuh", "sm100.cuh"],
     "decode_step": ["decode.cuh", "common.cuh"],
 }
 
@@ -425,6 +425,51 @@ def measure_config(name, dev, steps, warmup, peaks):
                     "decode_ms_per_step": dec_ms, "decode_frac_hbm": dec_gbs / peaks["hbm_gbs"],
                     "decode_alg_bytes_per_step": dec_bytes})
         del graph
+    return out
+
+
+def measure_fused(names, dev, steps, warmup, peaks):
+    """The fused prefill (ratp_prefill_fused: recurrence and attention in one
+    launch) beside the two-kernel path on the same inputs, timed with CUDA
+    events on the launching stream.  Reported beside the headline line."""
+    import recurrence_augmented_dilated_chunked_b200 as ratp
+    from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
+    out = {}
+    for name in names:
+        w = WORKLOADS[name]
+        stream = torch.cuda.current_stream(dev)
+        q, xk, xv, g = (t.to(dev) for t in prefill_inputs(w.B, w.T, w.H, w.Dh, w.dtype,
+                                                            w.gate_mean, w.gate_std, seed=0))
+        hk, hv, o = (torch.empty_like(q) for _ in range(3))
+        mask = w.dense_mask if w.dense_heads else None
+        ws = ratp.scan_workspace(w.B, w.T, w.H, w.Dh, q.dtype, dev)
+        fws = ratp.prefill_fused_workspace(w.B, w.T, w.H, w.Dh, dev)
+        runs = {
+            "fused": lambda: ratp.prefill_fused(q, xk, xv, g, w.D, w.W, head_mask=mask, hk=hk, hv=hv,
+                                                out=o, workspace=fws),
+            "two_kernel": lambda: (ratp.scan_prefill_kv(xk, xv, g, hk=hk, hv=hv, workspace=ws),
+                                   ratp.dilated_attn_prefill(q, hk, hv, w.D, w.W, head_mask=mask, out=o)),
+        }
+        r = {}
+        for key, run in runs.items():
+            evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+            for i in range(warmup + steps):
+                ev = evs[i - warmup] if i >= warmup else None
+                if ev:
+                    ev[0].record(stream)
+                run()
+                if ev:
+                    ev[1].record(stream)
+            torch.cuda.synchronize()
+            ratp.last_error(dev)
+            ms = statistics.median(e[0].elapsed_time(e[1]) for e in evs)
+            r[key] = {"ms": ms, "tokens_per_s": w.B * w.T / (ms / 1e3)}
+        # bytes the fused call must move: read q, x_k, x_v, g; write h_k, h_v, o
+        E = w.B * w.T * w.H * w.Dh
+        r["fused"]["alg_bytes"] = 7 * E * 2
+        r["fused"]["frac_hbm"] = 7 * E * 2 / (r["fused"]["ms"] / 1e3) / 1e9 / peaks["hbm_gbs"]
+        out[name] = r
+        del q, xk, xv, g, hk, hv, o
     return out
 
 
@@ -836,6 +881,8 @@ def run_ours(args, rank, world, local_rank):
         line["layer_stack_decode"] = measure_layer_stack(dev, min(args.steps, 5), args.warmup, peaks)
         line["per_sample_prefill"] = measure_per_sample("bf16_1p5b_T4096_D16", dev, min(args.steps, 5),
                                                         args.warmup, peaks)
+        line["fused_prefill"] = measure_fused([PREFILL, "bf16_1p5b_T4096_D16", "bf16_hybrid_7p6b_T8192_D4"],
+                                              dev, min(args.steps, 5), args.warmup, peaks)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = oracle_sample()
     print(json.dumps(line), flush=True)

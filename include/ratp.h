@@ -86,7 +86,7 @@ int ratp_device_sm_count(int* sms);
  *                            runs out;
  *   RATP_FAULT_FUSED_DROP_UNIT  the fused prefill never raises the done flag
  *                            of recurrence unit `arg` (unit = (b*H + h) *
- *                            ceil(T/256) + t/256), so the waits on it run out.
+ *                            ceil(T/128) + t/128), so the waits on it run out.
  * A wait that runs out ends its kernel early with RATP_ERR_TIMEOUT in the
  * device error word (outputs are then undefined); the context stays usable.
  * Returns RATP_ERR_ARG for an unknown kind, RATP_ERR_CUDA if the device
@@ -256,7 +256,7 @@ int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv
  * at position T-1 ([2][B][H][Dh], k then v; nullable), and o = attention of q
  * over hk, hv with dilation D, window W and head_mask (HOST array of H bytes,
  * nonzero = dense head; or NULL).  Inside the launch, scan warps compute the
- * recurrence 256 positions of one (b, h) at a time, ahead of the tensor-core
+ * recurrence 128 positions of one (b, h) at a time, ahead of the tensor-core
  * pipeline, which waits (bounded) on a per-unit flag before it loads keys a
  * unit holds; the recurrence runs in a different association order than
  * ratp_scan_prefill_kv, so results agree to rounding, not bit for bit.

@@ -198,14 +198,21 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
 }
 
 
-// Waits (whole warp) until every unit an item reads is scanned: the units
-// 0 .. (item's own) of its (b, h).  Then the TMA loads that lane 0 issues
-// next see the scan's stores.  False if the wait ran out or another CTA
-// aborted.
+// Waits (whole warp) until every unit holding a row that the item's tiles
+// load is scanned: units 0 up to the one with the last row of its last
+// window tile (up to 63 positions past its queries) or of its last dilated
+// tile (slots past the ones it attends to).  Rows a tile loads but no query
+// attends to still enter O += P V with P = 0, so they must hold finite values,
+// which an unscanned part of h_k/h_v need not.  Then the TMA loads that lane 0
+// issues next see the scan's stores.  False if the wait ran out or another
+// CTA aborted.
 __device__ __forceinline__ bool wait_units(const Params& p, const Item& it, unsigned int tag, int lane,
                                            volatile int* s_abort) {
   const long long first = ((long long)it.b * p.H + it.h) * p.NQ;
-  const int last = it.t0 / BM;
+  const int n_dt = it.n_tiles - it.n_win;                       // dilated (dense: positional) tiles
+  const long long win_end = it.n_win > 0 ? (long long)it.p_start + (long long)it.n_win * BN - 1 : 0;
+  const long long dil_end = (long long)n_dt * BN * it.Dd - 1;   // last row of the last dilated tile
+  const int last = (int)min((long long)p.NQ - 1, max(win_end, dil_end) / BM);
   const unsigned long long t0 = global_ns();
   unsigned int polls = 0;
   for (int j0 = 0; j0 <= last; j0 += 32) {

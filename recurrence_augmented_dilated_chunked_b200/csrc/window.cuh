@@ -24,10 +24,11 @@
 // both streams.  TMA stages the gate and the two inputs for rows
 // [t0 - 64, t0 + 256) (the 64-row halo holds the previous block of the
 // chunk's first block; rows before 0 or past T are filled with zeros, which
-// contribute nothing).  Warp w takes stream w % 2 and block lane w / 2; lane
-// = channel.  A thread runs the backward pass of the previous block (S in
-// registers, L of them) and the forward pass of its own block for blocks
-// lane, lane + 4, ... of the chunk.  No CTA depends on another: there is no
+// contribute nothing).  A thread owns a channel pair (bf16x2 or float2 loads
+// from shared memory, packed f32x2 arithmetic, 4- or 8-byte stores) of one
+// stream and runs, for blocks blane, blane + 4, ... of the chunk, the
+// backward pass of the previous block (S of both channels in registers) and
+// the forward pass of its own block.  No CTA depends on another: there is no
 // look-back and no workspace.  The one wait (the TMA tiles) is bounded.
 #pragma once
 #include "common.cuh"
@@ -36,7 +37,7 @@
 namespace ratp {
 namespace window {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 128;  // 16 channel pairs x 2 streams x 4 block lanes
 constexpr int kChunk = 256;    // tokens per CTA
 constexpr int kCh = 32;        // channels per CTA
 constexpr int kHalo = 64;      // rows staged before the chunk (>= L)
@@ -57,16 +58,19 @@ struct Params {
   int n_chunks_t;          // chunks along T
 };
 
-__device__ __forceinline__ float to_f(float v) { return v; }
-__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
-__device__ __forceinline__ void put(float* p, float v) { __stcs(p, v); }
-__device__ __forceinline__ void put(__nv_bfloat16* p, float v) {
-  __stcs(reinterpret_cast<unsigned short*>(p), __bfloat16_as_ushort(__float2bfloat16_rn(v)));
+// a channel pair of one staged row, as fp32
+__device__ __forceinline__ float2 ld_pair(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float2 ld_pair(const __nv_bfloat16* p) {
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ void st_pair(float* p, float2 v) { __stcs(reinterpret_cast<float2*>(p), v); }
+__device__ __forceinline__ void st_pair(__nv_bfloat16* p, float2 v) {
+  __stcs(reinterpret_cast<unsigned int*>(p), pack_bf16x2(v.x, v.y));
 }
 
-// Three CTAs per SM (61.5 KB of tiles each for bf16): the register cap of
-// 85 costs a few bytes of spill and measured 156 us at T=16K, L=64, against
-// 168 us with two CTAs per SM.
+// Three CTAs per SM (61.5 KB of tiles each for bf16), 128 threads each: a
+// thread keeps the L backward-pass sums of its two channels in registers.
 template <typename T, int L>
 __global__ void __launch_bounds__(kThreads, 3)
 window_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x0,
@@ -126,26 +130,26 @@ window_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ 
   }
 
   const T* sg = reinterpret_cast<const T*>(smem);
-  const int warp = tid >> 5, c = tid & 31;
-  const int s = warp & 1;                       // stream
-  const int bl = warp >> 1;                     // block lane
+  const int cp = 2 * (tid & 15);                // first channel of this thread's pair
+  const int s = (tid >> 4) & 1;                 // stream
+  const int bl = tid >> 5;                      // block lane
   const T* sx = reinterpret_cast<const T*>(smem + (1 + s) * SM::kTile);
-  T* out = p.h[s] + ((long long)b * p.Tn) * p.C + (long long)slab * kCh + c;
+  T* out = p.h[s] + ((long long)b * p.Tn) * p.C + (long long)slab * kCh + cp;
 
-  for (int k = bl; k < NB; k += kThreads / 64) {
+  for (int k = bl; k < NB; k += kThreads / 32) {
     const int cur = kHalo + k * L;              // smem row of the block start
     const int prev = cur - L;                   // smem row of the previous block
     // backward pass over the previous block: S[o] = its positions o+1 .. L-1
-    float S[L];
-    S[L - 1] = 0.f;
+    float2 S[L];
+    S[L - 1] = make_float2(0.f, 0.f);
     {
-      float suf = 0.f, P = 1.f;
+      float2 suf = make_float2(0.f, 0.f), P = make_float2(1.f, 1.f);
 #pragma unroll
       for (int o = L - 1; o >= 1; --o) {
-        const float gj = to_f(sg[(prev + o) * kCh + c]);
-        const float xj = to_f(sx[(prev + o) * kCh + c]);
-        suf = fmaf(P, fmaf(-gj, xj, xj), suf);
-        P *= gj;
+        const float2 gj = ld_pair(sg + (prev + o) * kCh + cp);
+        const float2 xj = ld_pair(sx + (prev + o) * kCh + cp);
+        suf = fma2(P, fma2(make_float2(-gj.x, -gj.y), xj, xj), suf);   // + P (1 - g) x
+        P = mul2(P, gj);
         S[o - 1] = suf;
       }
     }
@@ -153,16 +157,16 @@ window_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ 
     const int tb = t0 + k * L;                  // first token of the block
     T* dst = out + (long long)tb * p.C;
     const bool whole = tb + L <= p.Tn;          // warp-uniform: no per-token bound check
-    float loc = 0.f, A = 1.f;
+    float2 loc = make_float2(0.f, 0.f), A = make_float2(1.f, 1.f);
 #pragma unroll
     for (int o = 0; o < L; ++o) {
-      const float gj = to_f(sg[(cur + o) * kCh + c]);
-      const float xj = to_f(sx[(cur + o) * kCh + c]);
-      loc = fmaf(gj, loc - xj, xj);
-      A *= gj;
+      const float2 gj = ld_pair(sg + (cur + o) * kCh + cp);
+      const float2 xj = ld_pair(sx + (cur + o) * kCh + cp);
+      loc = fma2(gj, sub2(loc, xj), xj);
+      A = mul2(A, gj);
       if ((whole || tb + o < p.Tn) &&
-          RATP_IN((dst - p.h[s]), 1, (long long)p.B * p.Tn * p.C))
-        put(dst, fmaf(A, S[o], loc));
+          RATP_IN((dst - p.h[s]), 2, (long long)p.B * p.Tn * p.C))
+        st_pair(dst, fma2(A, S[o], loc));
       dst += p.C;
     }
   }

@@ -4,7 +4,7 @@ windowed, head-wise hybrid attention in one launch) against the oracle.
 The oracle runs the plain definitions in fp64: the sequential recurrence of
 each stream (oracle.scan) and softmax attention over the enumerated key sets
 (oracle.attention), on the same seeded inputs.  hk, hv, the final state and o
-are compared element by element on shapes that span several 256-position
+are compared element by element on shapes that span several 128-position
 units, ragged tails, D = 1, D >= T, windows shorter and longer than a tile
 and dense heads; at the full workload sizes on sampled rows and channels.
 """
@@ -40,8 +40,12 @@ CASES = [
 def _run(q, xk, xv, g, D, W, mask):
     B, T, H, Dh = q.shape
     fs = torch.zeros(2, B, H, Dh, dtype=torch.float32, device=DEV)
+    # h_k/h_v start as NaN: a key or value row read before its recurrence
+    # unit is scanned (even one whose softmax weight is 0) would show in o
+    hk = torch.full((B, T, H, Dh), float("nan"), dtype=q.dtype, device=DEV)
+    hv = torch.full_like(hk, float("nan"))
     o, hk, hv = ratp.prefill_fused(q.to(DEV), xk.to(DEV), xv.to(DEV), g.to(DEV), D, W, head_mask=mask,
-                                   final_state=fs)
+                                   hk=hk, hv=hv, final_state=fs)
     ratp.last_error()
     return o, hk, hv, fs
 
@@ -150,7 +154,7 @@ def test_fused_missing_unit_flag_times_out_then_recovers():
     q, xk, xv, g = (t.to(DEV) for t in prefill_inputs(B, T, H, 128, "bf16", seed=23))
     ratp.last_error()
     ratp.debug_fault(_binding.FAULT_SPIN_LIMIT, 20_000_000)
-    ratp.debug_fault(_binding.FAULT_FUSED_DROP_UNIT, 1)     # (b 0, h 0), positions 256..511
+    ratp.debug_fault(_binding.FAULT_FUSED_DROP_UNIT, 1)     # (b 0, h 0), positions 128..255
     try:
         ratp.prefill_fused(q, xk, xv, g, D, 0)
         with pytest.raises(RatpError, match="TIMEOUT"):
