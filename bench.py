@@ -657,7 +657,11 @@ def run_ours(args, rank, world, local_rank):
         mask = w.dense_mask if w.dense_heads else None
         L = w.D if args.variant == "chunk_local" else 0
         Ds = [1] * (w.B // 2) + [64] * (w.B - w.B // 2)
+        fws = ratp.prefill_fused_workspace(w.B, w.T, w.H, w.Dh, dev) if args.variant == "fused" else None
         for _ in range(args.warmup + args.steps):
+            if args.variant == "fused":
+                ratp.prefill_fused(q, xk, xv, g, w.D, w.W, head_mask=mask, hk=hk, hv=hv, out=o, workspace=fws)
+                continue
             if args.variant == "window":
                 ratp.scan_prefill_kv_window(xk, xv, g, 64, hk=hk, hv=hv)
             else:
@@ -903,10 +907,10 @@ def main():
                     help="run only this part, untimed (a driver for ncu captures)")
     ap.add_argument("--workload", default=None,
                     help="with --only prefill: the prefill workload (default: the headline one)")
-    ap.add_argument("--variant", choices=["chunk_local", "per_sample", "window"], default=None,
+    ap.add_argument("--variant", choices=["chunk_local", "per_sample", "window", "fused"], default=None,
                     help="with --only prefill: chunk-local scan (L = D), per-sample attention "
-                         "(first half of the batch dense, second half at D = 64), or the "
-                         "fixed look-back scan (L = 64)")
+                         "(first half of the batch dense, second half at D = 64), the "
+                         "fixed look-back scan (L = 64), or the fused prefill")
     args = ap.parse_args()
     if args.warmup < 3 and args.only is None:
         ap.error("--warmup must be >= 3")

@@ -84,15 +84,16 @@ int ratp_device_sm_count(int* sms);
  *   RATP_FAULT_ATTN_DROP_K   the first CTA of the tensor-core attention never
  *                            loads its K tile number `arg`, so the MMA's wait
  *                            runs out;
- *   RATP_FAULT_FUSED_DROP_UNIT  the fused prefill never raises the done flag
- *                            of recurrence unit `arg` (unit = (b*H + h) *
- *                            ceil(T/128) + t/128), so the waits on it run out.
+ *   RATP_FAULT_FUSED_DROP_CHUNK  the fused prefill never raises the done
+ *                            flag of scan chunk `arg` (chunk = (b * H*Dh/64
+ *                            + channel/64) * ceil(T/256) + t/256), so the
+ *                            waits on it run out.
  * A wait that runs out ends its kernel early with RATP_ERR_TIMEOUT in the
  * device error word (outputs are then undefined); the context stays usable.
  * Returns RATP_ERR_ARG for an unknown kind, RATP_ERR_CUDA if the device
  * update fails.  Not thread-safe with concurrent launches. */
 enum { RATP_FAULT_NONE = 0, RATP_FAULT_SPIN_LIMIT = 1, RATP_FAULT_SCAN_DROP = 2,
-       RATP_FAULT_ATTN_DROP_K = 3, RATP_FAULT_FUSED_DROP_UNIT = 4 };
+       RATP_FAULT_ATTN_DROP_K = 3, RATP_FAULT_FUSED_DROP_CHUNK = 4 };
 int ratp_debug_fault(int kind, long long arg);
 
 /* ------------------------------------------------------------------------
@@ -255,11 +256,14 @@ int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv
  * computes: hk = scan(xk, g), hv = scan(xv, g), final_state = the fp32 state
  * at position T-1 ([2][B][H][Dh], k then v; nullable), and o = attention of q
  * over hk, hv with dilation D, window W and head_mask (HOST array of H bytes,
- * nonzero = dense head; or NULL).  Inside the launch, scan warps compute the
- * recurrence 128 positions of one (b, h) at a time, ahead of the tensor-core
- * pipeline, which waits (bounded) on a per-unit flag before it loads keys a
- * unit holds; the recurrence runs in a different association order than
- * ratp_scan_prefill_kv, so results agree to rounding, not bit for bit.
+ * nonzero = dense head; or NULL).  Inside the launch, the CTAs that start
+ * first run the chunk scan of ratp_scan_prefill_kv (256 tokens x 64 channels
+ * per chunk, in sequence order) and raise a done flag per chunk; the others
+ * run the tensor-core attention over query tiles in ascending order and wait
+ * (bounded) for the flags of the chunks holding the rows they load.  The
+ * look-back of the scan composes a timing-dependent number of chunk maps,
+ * and the attention places its key tiles differently, so results agree with
+ * the two separate calls to rounding, not bit for bit.
  * q, xk, xv, g, hk, hv, o: [B][T][H][Dh] bf16, Dh = 128, device, 16-byte
  * aligned; hk and hv are written (they are outputs, and the attention reads
  * its keys back from them, mostly out of L2).

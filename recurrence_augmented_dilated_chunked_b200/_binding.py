@@ -375,7 +375,7 @@ def last_error(device=None):
     _check("ratp_last_error", lib.ratp_last_error(s))
 
 
-FAULT_NONE, FAULT_SPIN_LIMIT, FAULT_SCAN_DROP, FAULT_ATTN_DROP_K, FAULT_FUSED_DROP_UNIT = 0, 1, 2, 3, 4
+FAULT_NONE, FAULT_SPIN_LIMIT, FAULT_SCAN_DROP, FAULT_ATTN_DROP_K, FAULT_FUSED_DROP_CHUNK = 0, 1, 2, 3, 4
 
 
 def debug_fault(kind: int, arg: int = 0):

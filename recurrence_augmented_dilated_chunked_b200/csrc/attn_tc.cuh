@@ -56,6 +56,15 @@
 // Every mbarrier wait is bounded; on expiry the CTA records RATP_ERR_TIMEOUT,
 // all roles drain out (copies and MMAs in flight are waited for), and TMEM
 // is released.
+//
+// attn_kernel<true> is the fused prefill (fused.cuh): 256 threads per CTA;
+// the first CTAs to start scan the recurrence, the others run the pipeline
+// above (warps 6-7 idle) over query tiles in ascending order, waiting per
+// item for the scanned chunks it reads.  Its tiles end at the item's last
+// row: window tiles end at t_last and start at or before the window's first
+// row, the dilated tiles end at the item's last dilated slot (the first ones
+// may start before slot 0, which TMA fills with zeros), so no tile loads a
+// row after the item's last query.
 #pragma once
 #include "sm100.cuh"
 #include "fused.cuh"
@@ -71,11 +80,8 @@ constexpr int kSoftmaxWarps = 4;
 constexpr int kProducerWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kThreads = 192;
-// The fused prefill (recurrence and attention in one launch) adds two scan
-// warps per CTA (warps 6-7, fused.cuh) and their scratch.
-constexpr int kScanWarp0 = 6;
+// The fused prefill's CTAs have the chunk scan's 256 threads.
 constexpr int kThreadsFused = 256;
-constexpr uint32_t kScanScratch = 20 * 32 * 4;
 constexpr uint32_t kQHalf = BM * 64 * 2;       // Q: 128 rows x 64 columns: 16 KB
 constexpr uint32_t kQTile = 2 * kQHalf;        // 32 KB
 constexpr uint32_t kKHalf = BN * 64 * 2;       // K/V: 64 rows x 64 columns: 8 KB
@@ -84,11 +90,19 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffK = kOffQ + kQTile;     // 2 stages
 constexpr uint32_t kOffV = kOffK + 2 * kKTile; // 2 stages
 constexpr uint32_t kOffBar = kOffV + 2 * kKTile;
-// barriers: qfull qempty kfull[2] kempty[2] vfull[2] sfull sfree pfull[2] pvdone[2] final
-constexpr uint32_t kNumBars = 15;
-constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + TMEM slot, abort, tag, alignment
-constexpr uint32_t kOffScan = kOffBar + kNumBars * 8 + 16;               // fused: scan scratch
-constexpr uint32_t kSmemBytesFused = kSmemBytes + kScanScratch;
+// barriers: qfull qempty kfull[2] kempty[2] vfull[2] sfull sfree pfull[2] pvdone[2] final item[8]
+constexpr uint32_t kNumBars = 23;
+constexpr int kItemRing = 8;       // fused: item indices handed from the producer to the other roles
+// after the barriers: TMEM address, abort flag, item ring; then alignment slack
+constexpr uint32_t kCtlBytes = 8 + 4 * kItemRing;
+constexpr uint32_t kSmemBytes = kOffBar + kNumBars * 8 + kCtlBytes + 1024;
+// fused: a scan CTA stages its chunk tiles from the same (1024-aligned) base;
+// the barriers and control words lie past them, since the CTA goes on to
+// attend after its scan
+constexpr uint32_t kScanBytes = scan::Smem<__nv_bfloat16, 2>::kBytes;
+constexpr uint32_t kOffBarFused = (kScanBytes + 7) & ~7u;
+constexpr uint32_t kSmemBytesFused = kOffBarFused + kNumBars * 8 + kCtlBytes + 1024;
+static_assert(kOffBarFused >= kOffBar, "fused layout");
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0;      // S: 64 columns
 constexpr uint32_t kColP = 64;     // P buffer b at 64 + 32 b
@@ -136,18 +150,20 @@ struct Params {
   // fused prefill: items in ascending order (query tile major, then b, h),
   // head h dense where bit h of dense_bits is set, else dilation dil_D[0]
   unsigned long long dense_bits[RATP_MAX_HEADS / 64];
-  fused::ScanParams scan;
-  int tag_ctas;                    // CTAs of the launch (each draws the launch tag once)
+  fused::Scan scan;                // chunk scan of x_k, x_v with g into h_k, h_v
+  fused::Control ctl;
 };
 
-// The fused prefill's inputs x_k, x_v, g as [B][T][H][128] views (the L2
-// prefetch of the scan's next unit).
+// The fused prefill's scan inputs: [B][T][H*128] views of g, x_k, x_v, box
+// 64 channels x 256 tokens.
 struct ScanMaps {
-  CUtensorMap xk, xv, g;
+  CUtensorMap g, xk, xv;
 };
 
 struct Item {
   int b, h, t0, t_last, Dd, n_win, n_tiles, p_start, cls;
+  int win0;         // first row of the first window tile
+  int dil0;         // first slot of the first dilated tile (< 0: zero-filled rows)
   bool dense;
 };
 
@@ -190,55 +206,64 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
   } else {
     it.Dd = p.dil_D[it.cls];
     const int n_dil = max(0, it.t_last - p.W_eff + 1) / it.Dd;   // slots before the last row's window
+    const int n_dt = (n_dil + BN - 1) / BN;
     it.p_start = max(0, it.t0 - p.W_eff + 1);
     it.n_win = (it.t_last - it.p_start + 1 + BN - 1) / BN;
-    it.n_tiles = it.n_win + (n_dil + BN - 1) / BN;
+    it.n_tiles = it.n_win + n_dt;
+    // the fused prefill's tiles end at the item's last row / slot; the
+    // others start at the window's first row and at slot 0
+    it.win0 = FUSED ? it.t_last + 1 - it.n_win * BN : it.p_start;
+    it.dil0 = FUSED ? n_dil - n_dt * BN : 0;
+  }
+  if (it.dense) {
+    it.win0 = 0;
+    it.dil0 = 0;
   }
   return it;
 }
 
 
-// Waits (whole warp) until every unit holding a row that the item's tiles
-// load is scanned: units 0 up to the one with the last row of its last
-// window tile (up to 63 positions past its queries) or of its last dilated
-// tile (slots past the ones it attends to).  Rows a tile loads but no query
-// attends to still enter O += P V with P = 0, so they must hold finite values,
-// which an unscanned part of h_k/h_v need not.  Then the TMA loads that lane 0
-// issues next see the scan's stores.  False if the wait ran out or another
-// CTA aborted.
-__device__ __forceinline__ bool wait_units(const Params& p, const Item& it, unsigned int tag, int lane,
-                                           volatile int* s_abort) {
-  const long long first = ((long long)it.b * p.H + it.h) * p.NQ;
-  const int n_dt = it.n_tiles - it.n_win;                       // dilated (dense: positional) tiles
-  const long long win_end = it.n_win > 0 ? (long long)it.p_start + (long long)it.n_win * BN - 1 : 0;
-  const long long dil_end = (long long)n_dt * BN * it.Dd - 1;   // last row of the last dilated tile
-  const int last = (int)min((long long)p.NQ - 1, max(win_end, dil_end) / BM);
+// Waits (whole warp) until the scan has stored every row that the item's
+// tiles load: with the fused prefill's tile placement all of them lie at or
+// before t_last, and chunks complete in sequence order per chain, so the done
+// flags of t_last's chunk in the head's two 64-channel chains suffice (lanes
+// 0 and 1 poll one each).  Rows a tile loads but no query attends to still
+// enter O += P V with P = 0, so they must hold finite values, which an
+// unscanned part of h_k/h_v need not.  Then the TMA loads that lane 0 issues
+// next see the scan's stores.  False if the wait ran out or another CTA
+// aborted.
+__device__ __forceinline__ bool wait_chunks(const Params& p, const Item& it, unsigned int tag, int lane,
+                                            volatile int* s_abort) {
+  const fused::Scan& sc = p.scan;
+  const int chunk = min(it.t_last / scan::Shape<__nv_bfloat16>::kChunk, sc.n_chunks_t - 1);
+  const long long chain = (long long)it.b * sc.slabs + 2 * it.h + (lane & 1);
+  const long long desc = chain * sc.n_chunks_t + chunk;
   const unsigned long long t0 = global_ns();
   unsigned int polls = 0;
-  for (int j0 = 0; j0 <= last; j0 += 32) {
-    const int j = j0 + lane;
-    bool done = j > last;
-    while (true) {
-      if (!done && RATP_IN(first + j, 1, (long long)p.B * p.H * p.NQ))
-        done = fused::ld_acquire(p.scan.ws.flags + first + j) == tag;
-      if (__all_sync(0xffffffffu, done)) break;
-      bool give_up = false;
-      if ((++polls & 15u) == 0u)
-        give_up = *s_abort || fused::aborted(p.scan.ws) || global_ns() - t0 > spin_timeout();
-      if (__any_sync(0xffffffffu, give_up)) {
-        if (lane == 0) {
-          *s_abort = 1;
-          fused::abort_all(p.scan.ws);
-        }
-        return false;
-      }
-      __nanosleep(32);
+  bool done = lane >= 2;
+  while (true) {
+    if (!done && RATP_IN(desc, 1, (long long)sc.n_chains * sc.n_chunks_t))
+      done = fused::ld_acquire(sc.done + desc) == tag;
+    if (__all_sync(0xffffffffu, done)) break;
+    bool expired = false, give_up = false;
+    if ((++polls & 15u) == 0u) {
+      expired = global_ns() - t0 > spin_timeout();
+      give_up = expired || *s_abort || fused::aborted(sc.ws.abort);
     }
+    if (__any_sync(0xffffffffu, give_up)) {
+      if (__any_sync(0xffffffffu, expired) && lane == 0) raise_error(RATP_ERR_TIMEOUT);
+      if (lane == 0) {
+        *s_abort = 1;
+        fused::abort_all(sc.ws.abort);
+      }
+      return false;
+    }
+    __nanosleep(32);
   }
   __syncwarp();
   if (lane == 0) {
     asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    fused::fence_proxy_async_global();
+    asm volatile("fence.proxy.async.global;" ::: "memory");
   }
   __syncwarp();
   return true;
@@ -258,7 +283,8 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sb = smem_u32(smem);
   const uint32_t sQ = sb + kOffQ, sK = sb + kOffK, sV = sb + kOffV;
-  const uint32_t bar0 = sb + kOffBar;
+  constexpr uint32_t off_bar = FUSED ? kOffBarFused : kOffBar;
+  const uint32_t bar0 = sb + off_bar;
   const uint32_t b_qfull = bar0 + 0 * 8;    // Q landed
   const uint32_t b_qempty = bar0 + 1 * 8;   // last S = Q K^T of an item done
   const uint32_t b_kfull = bar0 + 2 * 8;    // [2] K stage landed
@@ -269,9 +295,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t b_pfull = bar0 + 10 * 8;   // [2] P buffer written (128 threads)
   const uint32_t b_pvdone = bar0 + 12 * 8;  // [2] O += P V done: P buffer and V stage free
   const uint32_t b_final = bar0 + 14 * 8;
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffBar + kNumBars * 8);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffBar + kNumBars * 8 + 4);
-  unsigned int* s_tag = reinterpret_cast<unsigned int*>(smem + kOffBar + kNumBars * 8 + 8);
+  const uint32_t b_item = bar0 + 15 * 8;    // [kItemRing] fused: item index written
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + off_bar + kNumBars * 8);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + off_bar + kNumBars * 8 + 4);
+  volatile int* s_items = reinterpret_cast<volatile int*>(smem + off_bar + kNumBars * 8 + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -289,10 +316,12 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(b_pvdone + 8 * i, 1);
     }
     mbar_init(b_final, 1);
+    for (int i = 0; i < kItemRing; ++i) mbar_init(b_item + 8 * i, 1);
     *s_abort = 0;
-    if (FUSED) *s_tag = fused::draw_tag(p.scan.ws, (unsigned int)p.tag_ctas);
     fence_barrier_init();
   }
+  // every CTA allocates its tensor memory and gives up the allocation permit
+  // at once (a fused scan CTA attends after its scan)
   if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(s_tmem), kTmemCols);
     tmem_relinquish();
@@ -306,30 +335,69 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       prefetch_tmap(&tm_dil.v[c]);
     }
   }
+  unsigned int tag = 0u;
+  __shared__ unsigned int s_start, s_tag;
+  if (FUSED && threadIdx.x == 0) {
+    // the role comes from the order in which the CTAs start (fused.cuh);
+    // every CTA draws exactly one ticket, which also returns the launch tag
+    unsigned int tk;
+    s_tag = scan::draw_ticket(p.scan.ws, (unsigned int)p.ctl.n_ctas, &tk);
+    s_start = tk;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const unsigned int tag = FUSED ? *s_tag : 0u;
+  if (FUSED) {
+    tag = s_tag;
+    if ((int)s_start < p.ctl.n_scan) {
+      // scan until the chunk tickets run out, then attend like the others
+      fused::scan_role(tm_scan.g, tm_scan.xk, tm_scan.xv, p.scan, p.ctl, smem, tag);
+      __syncthreads();
+    }
+  }
+  // This CTA's items: FUSED draws them one by one from the launch's item
+  // counter (ascending), the producer passing each index on through the ring
+  // (an index >= n_items ends the loop); otherwise blockIdx.x, +G, +2G, ...
+  // The producer runs at most a few items ahead of the MMA issuer and the
+  // softmax (it waits for O += P V of tile n-2 before it loads tile n), far
+  // less than the ring's depth.
+  auto item_at = [&](int li) -> int {
+    if (!FUSED) return (int)blockIdx.x + li * (int)gridDim.x;
+    if (!mbar_wait(b_item + 8 * (li % kItemRing), (uint32_t)(li / kItemRing) & 1u, s_abort)) return -1;
+    return s_items[li % kItemRing];
+  };
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     // Tile n (stage n%2): K once S = Q K^T of tile n-2 read the stage; at an
     // item's first tile then Q, once the previous item's last S = Q K^T is
     // done (its K load is already under way); V once O += P V of tile n-2
-    // read the stage.  The fused prefill first waits (whole warp) for the
-    // recurrence units the item reads.
-    int n = 0, li = 0, nq = 0;
+    // read the stage.  The fused prefill draws the item, passes its index on
+    // and first waits (whole warp) for the scanned chunks the item reads.
+    int n = 0, nq = 0;
     int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};   // last tile loaded per stage
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
+    for (int li = 0;; ++li) {
+      int idx;
+      if (FUSED) {
+        if (lane == 0) {
+          idx = ok ? (int)min(atomicAdd(p.ctl.items, 1u), (unsigned int)p.n_items) : p.n_items;
+          s_items[li % kItemRing] = idx;           // n_items: no more items
+          mbar_arrive(b_item + 8 * (li % kItemRing));
+        }
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+      } else {
+        idx = (int)blockIdx.x + li * (int)gridDim.x;
+      }
+      if (!ok || idx >= p.n_items) break;
       const Item it = make_item<FUSED>(p, idx);
-      if (FUSED && !wait_units(p, it, tag, lane, s_abort)) ok = false;
+      if (FUSED && !wait_chunks(p, it, tag, lane, s_abort)) ok = false;
       if (ok && lane == 0) {
         for (int j = 0; j < it.n_tiles; ++j, ++n) {
           const int st = n & 1;
           const bool pos = (j < it.n_win) || it.dense;
-          const int row = (j < it.n_win) ? it.p_start + j * BN : (j - it.n_win) * BN;
+          const int row = (j < it.n_win) ? it.win0 + j * BN : it.dil0 + (j - it.n_win) * BN;
           if (n >= 2 && !mbar_wait(b_kempty + 8 * st, ((n - 2) >> 1) & 1, s_abort)) { ok = false; break; }
           if (!(blockIdx.x == 0 && (long long)n == g_fault_attn_ktile)) {   // else: planted failure
             const CUtensorMap* m = pos ? &tm_kpos : &tm_dil.k[it.cls];
@@ -377,7 +445,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       const uint64_t dv0 = sw128_desc(sV, kKHalf, 1024);
       constexpr uint64_t kStageDesc = kKTile >> 4;      // descriptor step between stages
       const uint32_t tS = tmem + kColS, tP = tmem + kColP, tO = tmem + kColO;
-      int n = 0, li = 0;
+      int n = 0;
       bool ok = true;
       // S = Q K^T of tile n (its S columns were read by the softmax of n-1)
       auto issue_s = [&](int nn) -> bool {
@@ -411,7 +479,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         umma_commit(b_pvdone + 8 * st);
         return true;
       };
-      for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x, ++li) {
+      for (int li = 0; ok; ++li) {
+        const int idx = item_at(li);
+        if (idx < 0) { ok = false; break; }
+        if (idx >= p.n_items) break;
         const int n_tiles = make_item<FUSED>(p, idx).n_tiles;
         if (!mbar_wait(b_qfull, li & 1, s_abort)) { ok = false; break; }
         if (!issue_s(n)) { ok = false; break; }
@@ -439,7 +510,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     // always executed by the whole warp.
     int n = 0;                                       // tiles so far
     bool ok = true;
-    for (int idx = blockIdx.x; ok && idx < p.n_items; idx += gridDim.x) {
+    for (int li = 0; ok; ++li) {
+      const int idx = item_at(li);
+      if (!warp_all(idx >= 0)) { ok = false; break; }
+      if (idx >= p.n_items) break;
       const Item it = make_item<FUSED>(p, idx);
       const int t = it.t0 + r;
       const int lim_dil = it.dense ? (t + 1) : (max(0, t - p.W_eff + 1) / it.Dd);
@@ -459,12 +533,13 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         // valid columns [lo, hi) of this row in this tile, as 32-bit chunk masks
         int lo, hi;
         if (j < it.n_win) {
-          const int base = it.p_start + j * BN;
+          const int base = it.win0 + j * BN;
           lo = w_lo - base;
           hi = t - base + 1;
         } else {
-          lo = 0;
-          hi = lim_dil - (j - it.n_win) * BN;
+          const int base = it.dil0 + (j - it.n_win) * BN;   // < 0: leading zero-filled slots
+          lo = -base;
+          hi = lim_dil - base;
         }
         uint32_t vm[2];
 #pragma unroll
@@ -585,30 +660,6 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
       }
       tc_fence_before();
-    }
-  }
-
-  if (FUSED && warp >= kScanWarp0) {
-    // ------------------------------------------------------------ scan (fused prefill)
-    // This CTA's items in its own order, each item's unit scanned ahead of
-    // its attention; lane 0 of the first scan warp prefetches the next unit's
-    // inputs into L2.
-    const int sw = warp - kScanWarp0;
-    float* s_map = reinterpret_cast<float*>(smem + kOffScan);
-    for (int idx = blockIdx.x; idx < p.n_items; idx += gridDim.x) {
-      const Item it = make_item<FUSED>(p, idx);
-      if (sw == 0 && lane == 0 && idx + (int)gridDim.x < p.n_items) {
-        const Item nx = make_item<FUSED>(p, idx + gridDim.x);
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tma_prefetch_l2_4d(&tm_scan.g, 64 * c, nx.h, nx.t0, nx.b);
-          tma_prefetch_l2_4d(&tm_scan.xk, 64 * c, nx.h, nx.t0, nx.b);
-          tma_prefetch_l2_4d(&tm_scan.xv, 64 * c, nx.h, nx.t0, nx.b);
-        }
-      }
-      // a unit whose wait ran out still publishes (a zero carry), so that no
-      // other CTA waits on it; the error word holds the timeout
-      fused::scan_unit(p.scan, p.B, p.T, p.H, it.b, it.h, it.t0 / BM, sw, lane, tag, s_map, 1);
     }
   }
 

@@ -46,7 +46,7 @@ constexpr unsigned long long kSpinTimeoutNs = 2000000000ull;
 __device__ unsigned long long g_spin_timeout_ns = kSpinTimeoutNs;
 __device__ long long g_fault_scan_ticket = -1;    // scan chunk that publishes nothing
 __device__ long long g_fault_attn_ktile = -1;     // K tile the first attention CTA skips
-__device__ long long g_fault_fused_unit = -1;     // fused prefill unit whose done flag is never raised
+__device__ long long g_fault_fused_chunk = -1;    // fused prefill scan chunk whose done flag is never raised
 
 __device__ __forceinline__ unsigned long long spin_timeout() { return g_spin_timeout_ns; }
 

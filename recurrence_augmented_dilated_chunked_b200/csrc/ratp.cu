@@ -391,7 +391,16 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
 }
 
 // Fused prefill: the recurrence of both streams and the attention in one
-// launch (attn_kernel<true>: scan warps ahead of the tensor-core pipeline).
+// launch (attn_kernel<true>: scan CTAs and attention CTAs, fused.cuh).
+// Share of the launch's CTAs (two per SM) that scan first, in thousandths.
+// An SM shared by a scan CTA and an attention CTA runs each at about half
+// its two-CTA rate, so overlap gains little; most CTAs scan first, and the
+// rest start the attention on the sequence's first tiles (measured at
+// T = 16K: 500 -> 335 us, 700 -> 332 us, 850 -> 323 us, 1000 -> 326 us).
+#ifndef RATP_FUSED_SCAN_PER_MILLE
+#define RATP_FUSED_SCAN_PER_MILLE 850
+#endif
+
 int launch_prefill_fused(const void* q, const void* xk, const void* xv, const void* g, void* hk, void* hv,
                          void* o, float* fs, int B, int T, int H, int D, int W, const uint8_t* head_mask,
                          void* ws, size_t ws_bytes, cudaStream_t st) {
@@ -400,33 +409,47 @@ int launch_prefill_fused(const void* q, const void* xk, const void* xv, const vo
   p.o = static_cast<__nv_bfloat16*>(o);
   p.B = B; p.T = T; p.H = H; p.W_eff = W > 0 ? W : 1;
   p.NQ = (T + attn_tc::BM - 1) / attn_tc::BM;
-  const long long n_units = (long long)B * H * p.NQ;
-  if (n_units > 0x7fffffffll) return RATP_ERR_SHAPE;
-  if (ws_bytes < fused::workspace_bytes(n_units)) return RATP_ERR_CAPACITY;
-  int rc = read_mask(head_mask, H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
+  const long long n_items = (long long)B * H * p.NQ;
+  ScanGeom geo;
+  int rc = scan_geom(B, T, H, 128, RATP_BF16, &geo);
   if (rc) return rc;
-  p.n_items = (int)n_units;
+  if (n_items > 0x7fffffffll) return RATP_ERR_SHAPE;
+  if (ws_bytes < fused::workspace_bytes(geo.n_chunks)) return RATP_ERR_CAPACITY;
+  rc = read_mask(head_mask, H, p.dense_bits, nullptr, nullptr, nullptr, nullptr);
+  if (rc) return rc;
+  p.n_items = (int)n_items;
   p.n_cls = D > 1 ? 1 : 0;
   p.dil_D[0] = D;
   p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
-  p.scan.xk = static_cast<const __nv_bfloat16*>(xk);
-  p.scan.xv = static_cast<const __nv_bfloat16*>(xv);
-  p.scan.g = static_cast<const __nv_bfloat16*>(g);
-  p.scan.hk = static_cast<__nv_bfloat16*>(hk);
-  p.scan.hv = static_cast<__nv_bfloat16*>(hv);
+  fused::carve(ws, geo.n_chunks, &p.ctl, &p.scan);
+  p.scan.h[0] = static_cast<__nv_bfloat16*>(hk);
+  p.scan.h[1] = static_cast<__nv_bfloat16*>(hv);
   p.scan.final_state = fs;
-  p.scan.ws = fused::carve(ws, n_units);
-  p.scan.NQ = p.NQ;
+  p.scan.B = B; p.scan.Tn = T; p.scan.C = H * 128;
+  p.scan.reset_L = 0;
+  p.scan.slabs = geo.slabs; p.scan.n_chains = geo.n_chains; p.scan.n_chunks_t = geo.n_chunks_t;
+  // CTAs: two per SM; n_scan of them scan first (no more than there are
+  // chunks), and no more CTAs than the scan CTAs plus one per item
+  const int slots = attn_tc::kCtasPerSm * sm_count();
+  long long n_scan = ((long long)slots * RATP_FUSED_SCAN_PER_MILLE + 500) / 1000;
+  n_scan = std::max(1ll, std::min(n_scan, std::min(geo.n_chunks, (long long)slots - 1)));
+  const long long n_attn = std::min(n_items, (long long)slots - n_scan);
+  p.ctl.n_scan = (int)n_scan;
+  p.ctl.n_ctas = (int)(n_scan + n_attn);
+  p.scan.l2_ahead = (int)n_scan;   // one chunk per scan CTA ahead
   const long long row = (long long)H * 128, bat = (long long)T * row;
   constexpr int qr = attn_tc::BM, kr = attn_tc::BN;
+  constexpr int sr = scan::Shape<__nv_bfloat16>::kChunk;
   CUtensorMap tq, tkp, tvp;
   attn_tc::DilMaps dm;
   attn_tc::ScanMaps sm;
   memset(&dm, 0, sizeof(dm));
   if (!make_map(&tq, q, 0, B, T, H, row, bat, qr) || !make_map(&tkp, hk, 0, B, T, H, row, bat, kr) ||
-      !make_map(&tvp, hv, 0, B, T, H, row, bat, kr) || !make_map(&sm.xk, xk, 0, B, T, H, row, bat, qr) ||
-      !make_map(&sm.xv, xv, 0, B, T, H, row, bat, qr) || !make_map(&sm.g, g, 0, B, T, H, row, bat, qr))
+      !make_map(&tvp, hv, 0, B, T, H, row, bat, kr) ||
+      !make_scan_map<__nv_bfloat16>(&sm.g, g, B, T, H * 128, sr) ||
+      !make_scan_map<__nv_bfloat16>(&sm.xk, xk, B, T, H * 128, sr) ||
+      !make_scan_map<__nv_bfloat16>(&sm.xv, xv, B, T, H * 128, sr))
     return RATP_ERR_CUDA;
   const long long n_slots = D > 1 ? T / D : 0;
   if (n_slots >= 1) {
@@ -439,12 +462,9 @@ int launch_prefill_fused(const void* q, const void* xk, const void* xv, const vo
   }
   auto kernel = attn_tc::attn_kernel<true>;
   if (!ensure_smem(kernel, (int)attn_tc::kSmemBytesFused)) return RATP_ERR_CUDA;
-  const int slots = attn_tc::kCtasPerSm * sm_count();
-  const int grid = p.n_items < slots ? p.n_items : slots;
-  p.tag_ctas = grid;
   if (cudaMemsetAsync(static_cast<char*>(ws) + fused::kResetOffset, 0, fused::kResetBytes, st) != cudaSuccess)
     return RATP_ERR_CUDA;
-  kernel<<<grid, attn_tc::kThreadsFused, attn_tc::kSmemBytesFused, st>>>(tq, tkp, tvp, dm, sm, p);
+  kernel<<<p.ctl.n_ctas, attn_tc::kThreadsFused, attn_tc::kSmemBytesFused, st>>>(tq, tkp, tvp, dm, sm, p);
   return launch_status();
 }
 
@@ -594,7 +614,7 @@ int ratp_debug_fault(int kind, long long arg) {
       ok = cudaMemcpyToSymbol(ratp::g_spin_timeout_ns, &timeout, sizeof(timeout)) == cudaSuccess &&
            cudaMemcpyToSymbol(ratp::g_fault_scan_ticket, &none, sizeof(none)) == cudaSuccess &&
            cudaMemcpyToSymbol(ratp::g_fault_attn_ktile, &none, sizeof(none)) == cudaSuccess &&
-           cudaMemcpyToSymbol(ratp::g_fault_fused_unit, &none, sizeof(none)) == cudaSuccess;
+           cudaMemcpyToSymbol(ratp::g_fault_fused_chunk, &none, sizeof(none)) == cudaSuccess;
       break;
     case RATP_FAULT_SPIN_LIMIT:
       ok = cudaMemcpyToSymbol(ratp::g_spin_timeout_ns, &timeout, sizeof(timeout)) == cudaSuccess;
@@ -605,8 +625,8 @@ int ratp_debug_fault(int kind, long long arg) {
     case RATP_FAULT_ATTN_DROP_K:
       ok = cudaMemcpyToSymbol(ratp::g_fault_attn_ktile, &arg, sizeof(arg)) == cudaSuccess;
       break;
-    case RATP_FAULT_FUSED_DROP_UNIT:
-      ok = cudaMemcpyToSymbol(ratp::g_fault_fused_unit, &arg, sizeof(arg)) == cudaSuccess;
+    case RATP_FAULT_FUSED_DROP_CHUNK:
+      ok = cudaMemcpyToSymbol(ratp::g_fault_fused_chunk, &arg, sizeof(arg)) == cudaSuccess;
       break;
     default:
       return RATP_ERR_ARG;
@@ -733,9 +753,10 @@ int ratp_dilated_attn_prefill(const void* q, const void* hk, const void* hv, voi
 int ratp_prefill_fused_workspace_bytes(int B, int T, int H, int Dh, size_t* bytes) {
   if (!bytes || B < 0 || T < 0 || H < 0) return RATP_ERR_ARG;
   if (Dh != 128) return RATP_ERR_UNSUPPORTED;
-  const long long n_units = (long long)B * H * ((T + attn_tc::BM - 1) / attn_tc::BM);
-  if (n_units > 0x7fffffffll) return RATP_ERR_SHAPE;
-  *bytes = fused::workspace_bytes(n_units);
+  ScanGeom geo;
+  const int rc = scan_geom(B, T, H, 128, RATP_BF16, &geo);
+  if (rc) return rc;
+  *bytes = fused::workspace_bytes(geo.n_chunks);
   return RATP_OK;
 }
 

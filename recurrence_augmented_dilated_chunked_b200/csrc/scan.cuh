@@ -163,6 +163,7 @@ struct Params {
   int slabs;              // C / 64
   int n_chains;           // B * slabs
   int n_chunks_t;         // chunks along T
+  unsigned int* done;     // fused prefill only: per-chunk done flags (see scan_chunk)
 };
 
 // Dynamic shared memory: (1 + NS) tiles of [chunk][64] elements filled by TMA
@@ -175,21 +176,28 @@ struct Smem {
   static constexpr int kBytes = kData + kScan + 128;                       // + alignment
 };
 
-template <typename T, int NS, int R = kRows, bool RESET = false>
-__global__ void __launch_bounds__(kThreads, 2)
-scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x0,
-            const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ Params<T, NS> p) {
+// One chunk (the chunk of `ticket`) by the whole CTA: its tiles are staged
+// into `smem` (128-byte aligned, Smem::kBytes) through the mbarrier `bar`,
+// whose phase `parity` this call completes.  Returns false when a bounded
+// wait ran out or another CTA aborted; a CTA that goes on using `smem` must
+// then first let the copies in flight on `bar` land.
+// FUSED (the fused prefill, whose attention reads h_k/h_v right after the
+// scan): the stores keep their lines in L2 (no streaming hint), and once all
+// of the chunk is stored, after its predecessor in the chain, the chunk's done
+// flag p.done[desc] takes the launch tag.  Flags therefore complete in
+// sequence order per chain: a reader that sees chunk c done may read every
+// row of the chain up to the end of chunk c.
+template <typename T, int NS, int R, bool RESET, bool FUSED>
+__device__ __forceinline__ bool scan_chunk(const CUtensorMap& tm_g, const CUtensorMap& tm_x0,
+                                           const CUtensorMap& tm_x1, const Params<T, NS>& p, uint8_t* smem,
+                                           uint32_t bar, uint32_t parity, unsigned int ticket, unsigned int tag) {
   using S = Shape<T, R>;
   using SM = Smem<T, NS, R>;
   constexpr int V = S::kVec, V2 = V / 2, LANES = S::kLanes, L = S::kChunk;
   constexpr int NW = kThreads / 32;
 
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const T* s_g = reinterpret_cast<const T*>(smem);
   float* s_w = reinterpret_cast<float*>(smem + SM::kData);            // [NW][1 + NS][64]
-  __shared__ __align__(8) uint64_t s_bar;
-  __shared__ unsigned int s_ticket, s_tag;
   __shared__ float s_tot_a[kSlab];
   __shared__ float s_tot_b[NS][kSlab];
   __shared__ float s_carry[NS][kSlab];
@@ -201,17 +209,6 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p.ws.abort) : "memory");
     return v != 0u;
   };
-  const uint32_t bar = sm100::smem_u32(&s_bar);
-  if (tid == 0) {
-    unsigned int tk;
-    s_tag = draw_ticket(p.ws, (unsigned int)(p.n_chains * p.n_chunks_t), &tk);
-    s_ticket = tk;
-    sm100::mbar_init(bar, 1);
-    sm100::fence_barrier_init();
-  }
-  __syncthreads();
-  const unsigned int ticket = s_ticket;
-  const unsigned int tag = s_tag;
   const int chunk = ticket / p.n_chains;     // chunk-major: predecessors started earlier
   const int chain = ticket % p.n_chains;
   const int b = chain / p.slabs;
@@ -259,7 +256,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
     if (tid == 0) {
       unsigned long long tw = 0;
       unsigned int n = 0;
-      while (!sm100::mbar_try_wait(bar, 0)) {
+      while (!sm100::mbar_try_wait(bar, parity)) {
         if ((++n & 63u) == 0u) {
           const unsigned long long now = global_ns();
           if (tw == 0) tw = now;
@@ -279,7 +276,7 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
           atomicExch(p.ws.abort, 1u);
         }
       }
-      return;
+      return false;
     }
   }
 
@@ -564,8 +561,10 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
 #pragma unroll
         for (int i = 0; i < V2; ++i) hs[s][i] = fma2(gf[i], sub2(hs[s][i], xf[i]), xf[i]);
         const long long off = base + (long long)t * row_stride;
-        if (RATP_IN(off, V, (long long)p.B * p.Tn * p.C))
-          __stcs(reinterpret_cast<uint4*>(p.h[s] + off), Elem<T>::pack2(hs[s]));
+        if (RATP_IN(off, V, (long long)p.B * p.Tn * p.C)) {
+          if (FUSED) *reinterpret_cast<uint4*>(p.h[s] + off) = Elem<T>::pack2(hs[s]);
+          else __stcs(reinterpret_cast<uint4*>(p.h[s] + off), Elem<T>::pack2(hs[s]));
+        }
         if (t == p.Tn - 1 && p.final_state != nullptr &&
             RATP_IN(((long long)s * p.B + b) * p.C + slab * kSlab + lane_c * V, V, (long long)NS * p.B * p.C)) {
           float* fs = p.final_state + ((long long)s * p.B + b) * p.C + slab * kSlab + lane_c * V;
@@ -574,6 +573,66 @@ scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CU
         }
       }
     }
+  }
+  if (!FUSED) return true;
+
+  // ---- done flag (fused prefill) ----
+  // Every thread orders its stores before the attention's TMA reads (async
+  // proxy); after the barrier thread 0 waits (bounded) for the predecessor's
+  // flag and releases this chunk's.
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __syncthreads();
+  bool ok = true;
+  if (tid == 0) {
+    [[maybe_unused]] const long long n_desc = (long long)p.n_chains * p.n_chunks_t;
+    if (chunk > 0) {
+      const unsigned int* prev = p.done + desc - 1;
+      const unsigned long long t_start = global_ns();
+      unsigned int v = 0u;
+      while (true) {
+        if (RATP_IN(desc - 1, 1, n_desc))
+          asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(prev) : "memory");
+        if (v == tag) break;
+        if (global_ns() - t_start > spin_timeout() || aborted()) {
+          raise_error(RATP_ERR_TIMEOUT);
+          atomicExch(p.ws.abort, 1u);
+          ok = false;
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
+    if (ok && desc != g_fault_fused_chunk && RATP_IN(desc, 1, n_desc)) {   // else: planted failure
+      __threadfence();
+      asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p.done + desc), "r"(tag) : "memory");
+    }
+  }
+  return __syncthreads_and(ok) != 0;
+}
+
+template <typename T, int NS, int R = kRows, bool RESET = false>
+__global__ void __launch_bounds__(kThreads, 2)
+scan_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_x0,
+            const __grid_constant__ CUtensorMap tm_x1, const __grid_constant__ Params<T, NS> p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  __shared__ __align__(8) uint64_t s_bar;
+  __shared__ unsigned int s_ticket, s_tag;
+  const uint32_t bar = sm100::smem_u32(&s_bar);
+  if (threadIdx.x == 0) {
+    unsigned int tk;
+    s_tag = draw_ticket(p.ws, (unsigned int)(p.n_chains * p.n_chunks_t), &tk);
+    s_ticket = tk;
+    sm100::mbar_init(bar, 1);
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  // one chunk per CTA; after a failed wait, the copies still in flight land
+  // (bounded) before the CTA's shared memory is released
+  if (!scan_chunk<T, NS, R, RESET, false>(tm_g, tm_x0, tm_x1, p, smem, bar, 0u, s_ticket, s_tag) &&
+      threadIdx.x == 0) {
+    const unsigned long long t1 = global_ns();
+    while (!sm100::mbar_try_wait(bar, 0) && global_ns() - t1 < spin_timeout()) {}
   }
 }
 

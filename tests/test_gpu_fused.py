@@ -4,9 +4,10 @@ windowed, head-wise hybrid attention in one launch) against the oracle.
 The oracle runs the plain definitions in fp64: the sequential recurrence of
 each stream (oracle.scan) and softmax attention over the enumerated key sets
 (oracle.attention), on the same seeded inputs.  hk, hv, the final state and o
-are compared element by element on shapes that span several 128-position
-units, ragged tails, D = 1, D >= T, windows shorter and longer than a tile
-and dense heads; at the full workload sizes on sampled rows and channels.
+are compared element by element on shapes that span several 256-token scan
+chunks and 128-query tiles, ragged tails, D = 1, D >= T, windows shorter and
+longer than a key tile and dense heads; at the full workload sizes on sampled
+rows and channels.
 """
 import numpy as np
 import pytest
@@ -149,12 +150,12 @@ def test_fused_argument_errors():
     ratp.last_error()
 
 
-def test_fused_missing_unit_flag_times_out_then_recovers():
+def test_fused_missing_chunk_flag_times_out_then_recovers():
     B, T, H, D = 1, 1000, 2, 4
     q, xk, xv, g = (t.to(DEV) for t in prefill_inputs(B, T, H, 128, "bf16", seed=23))
     ratp.last_error()
     ratp.debug_fault(_binding.FAULT_SPIN_LIMIT, 20_000_000)
-    ratp.debug_fault(_binding.FAULT_FUSED_DROP_UNIT, 1)     # (b 0, h 0), positions 128..255
+    ratp.debug_fault(_binding.FAULT_FUSED_DROP_CHUNK, 1)    # b 0, channels 0..63, positions 256..511
     try:
         ratp.prefill_fused(q, xk, xv, g, D, 0)
         with pytest.raises(RatpError, match="TIMEOUT"):
