@@ -167,7 +167,7 @@ class ClockSampler:
 
 KERNEL_SOURCES = {
     "scan_kv": ["scan.cuh", "common.cuh", "sm100.cuh"],
-    "dilated_attn": ["attn_tc.cuh", "fused.cuh", "common.cuh", "sm100.cuh"],
+    "dilated_attn": ["attn_tc.cuh", "fused.cuh", "scan.cuh", "common.cuh", "sm100.cuh"],
     "decode_step": ["decode.cuh", "common.cuh"],
 }
 

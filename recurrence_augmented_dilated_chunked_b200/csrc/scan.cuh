@@ -113,12 +113,6 @@ inline Workspace carve(void* base, long long n_chunks, int NS) {
 // Zeroed before each launch: the abort word (the ticket word is kept).
 constexpr size_t kResetOffset = 128, kResetBytes = 64;
 
-// L2 prefetch of one tile of a 3-D tensor map (no shared-memory destination).
-__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
-               :: "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2) : "memory");
-}
-
 __device__ __forceinline__ void put_word(unsigned long long* p, float v, unsigned int tag) {
   const unsigned long long w = ((unsigned long long)tag << 32) | __float_as_uint(v);
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(w) : "memory");
@@ -229,9 +223,9 @@ __device__ __forceinline__ bool scan_chunk(const CUtensorMap& tm_g, const CUtens
       if (p.l2_ahead > 0 && nt < (long long)p.n_chains * p.n_chunks_t) {
         const int ck = (int)(nt / p.n_chains), chn = (int)(nt % p.n_chains);
         const int b2 = chn / p.slabs, s2 = chn % p.slabs;
-        tma_prefetch_l2_3d(&tm_g, s2 * kSlab, ck * L, b2);
-        tma_prefetch_l2_3d(&tm_x0, s2 * kSlab, ck * L, b2);
-        if (NS == 2) tma_prefetch_l2_3d(&tm_x1, s2 * kSlab, ck * L, b2);
+        sm100::tma_prefetch_l2_3d(&tm_g, s2 * kSlab, ck * L, b2);
+        sm100::tma_prefetch_l2_3d(&tm_x0, s2 * kSlab, ck * L, b2);
+        if (NS == 2) sm100::tma_prefetch_l2_3d(&tm_x1, s2 * kSlab, ck * L, b2);
       }
     }
   }

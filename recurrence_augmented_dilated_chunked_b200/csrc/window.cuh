@@ -30,6 +30,8 @@
 // backward pass of the previous block (S of both channels in registers) and
 // the forward pass of its own block.  No CTA depends on another: there is no
 // look-back and no workspace.  The one wait (the TMA tiles) is bounded.
+// Thread 0 also prefetches into L2 the tiles of the CTA one SM count of
+// blocks later, so that the loads of later CTAs mostly hit L2.
 #pragma once
 #include "common.cuh"
 #include "sm100.cuh"
@@ -56,6 +58,7 @@ struct Params {
   int B, Tn, C;            // Tn tokens, C = H * Dh channels per token
   int slabs;               // C / 32
   int n_chunks_t;          // chunks along T
+  int l2_ahead;            // L2 prefetch distance in CTAs (0: none)
 };
 
 // a channel pair of one staged row, as fp32
@@ -104,6 +107,20 @@ window_kernel(const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ 
       for (int r = 0; r < kRows / kBox; ++r)   // rows t0 - 64 + 64 r (the first box may start before 0)
         sm100::tma_load_3d(dst + m * SM::kTile + r * kBox * kCh * (int)sizeof(T), maps[m], bar,
                            slab * kCh, t0 - kHalo + r * kBox, b);
+    // warm L2 with the chunk of the CTA l2_ahead blocks later (its halo is
+    // this range's tail, fetched already), so that DRAM keeps streaming
+    // while the resident CTAs compute
+    const long long nb = (long long)blockIdx.x + p.l2_ahead;
+    if (p.l2_ahead > 0 && nb < (long long)p.B * p.slabs * p.n_chunks_t) {
+      const int ck = (int)(nb % p.n_chunks_t);
+      const long long rs = nb / p.n_chunks_t;
+      const int sl = (int)(rs % p.slabs), bb = (int)(rs / p.slabs);
+#pragma unroll
+      for (int m = 0; m < 3; ++m)
+#pragma unroll
+        for (int r = 1; r < kRows / kBox; ++r)
+          sm100::tma_prefetch_l2_3d(maps[m], sl * kCh, ck * kChunk - kHalo + r * kBox, bb);
+    }
   }
   bool ok = true;
   if (tid == 0) {
