@@ -90,6 +90,36 @@ def test_scan_workspace_query(lib):
     assert lib.ratp_scan_workspace_bytes(1, 10, 1, 64, 7, ctypes.byref(n)) == 1
 
 
+def test_fused_prefill_workspace_query(lib):
+    n = ctypes.c_size_t()
+    assert lib.ratp_prefill_fused_workspace_bytes(2, 16384, 16, 128, ctypes.byref(n)) == 0
+    # 256-token x 64-channel chunks: a 4-byte done flag each, plus the chunk
+    # scan's descriptor words for two streams (as ratp_scan_workspace_bytes)
+    chunks = 2 * (2048 // 64) * (16384 // 256)
+    s = ctypes.c_size_t()
+    assert lib.ratp_scan_workspace_bytes(2, 16384, 16, 128, 1, ctypes.byref(s)) == 0
+    assert n.value >= s.value + 4 * chunks
+    # a ragged T rounds the chunks up
+    m = ctypes.c_size_t()
+    assert lib.ratp_prefill_fused_workspace_bytes(1, 257, 2, 128, ctypes.byref(m)) == 0
+    assert m.value >= 4 * (1 * 4 * 2)
+    assert lib.ratp_prefill_fused_workspace_bytes(1, 256, 2, 64, ctypes.byref(m)) == 7    # Dh != 128
+    assert lib.ratp_prefill_fused_workspace_bytes(-1, 256, 2, 128, ctypes.byref(m)) == 1
+
+
+def test_fused_prefill_rejects_bad_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)
+    ws = ctypes.c_void_p(4096)
+    # null pointers, misalignment, fp32, too small a workspace, bad D / W
+    assert lib.ratp_prefill_fused(p, p, p, p, p, p, p, None, 1, 8, 1, 128, 4, 0, None, 1, None, 0, None) == 1
+    assert lib.ratp_prefill_fused(p, p, p, ctypes.c_void_p(18), p, p, p, None, 1, 8, 1, 128, 4, 0, None, 1,
+                                  ws, 1 << 20, None) == 3
+    assert lib.ratp_prefill_fused(p, p, p, p, p, p, p, None, 1, 8, 1, 128, 4, 0, None, 0, ws, 1 << 20, None) == 7
+    assert lib.ratp_prefill_fused(p, p, p, p, p, p, p, None, 1, 8, 1, 128, 4, 0, None, 1, ws, 16, None) == 4
+    assert lib.ratp_prefill_fused(p, p, p, p, p, p, p, None, 1, 8, 1, 128, 0, 0, None, 1, ws, 1 << 20, None) == 1
+    assert lib.ratp_prefill_fused(p, p, p, p, p, p, p, None, 1, 8, 1, 128, 4, -1, None, 1, ws, 1 << 20, None) == 1
+
+
 def test_cache_bytes_query(lib):
     n = ctypes.c_size_t()
     assert lib.ratp_cache_bytes(64, 16, 128, 33024, 64, 128, None, ctypes.byref(n)) == 0
