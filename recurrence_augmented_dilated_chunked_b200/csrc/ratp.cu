@@ -361,6 +361,7 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
   if (items > 0x7fffffffll) return RATP_ERR_SHAPE;
   p.n_items = (int)items;
   if (p.n_items == 0) return RATP_OK;
+  p.alternate = p.n_seg > 1;
   p.scale_log2 = 1.4426950408889634f / sqrtf(128.f);
   p.o_align32 = (reinterpret_cast<uintptr_t>(o) & 31u) == 0;
   const long long row = (long long)H * 128, bat = (long long)T * row;

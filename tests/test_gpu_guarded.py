@@ -17,7 +17,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 SMALL_TESTS = ["tests/test_gpu_scan.py", "tests/test_gpu_chunk_local.py", "tests/test_gpu_window.py",
                "tests/test_gpu_attn.py", "tests/test_gpu_per_sample.py", "tests/test_gpu_decode.py",
-               "tests/test_gpu_layers.py"]
+               "tests/test_gpu_layers.py", "tests/test_gpu_fused.py"]
 
 
 def _env(**extra):
