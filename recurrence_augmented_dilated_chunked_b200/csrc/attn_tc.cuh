@@ -28,9 +28,9 @@
 // for the whole batch (the per-head hybrid) is the case of a single dilated
 // segment; several (per-sample D, the batch composition of the write-up's
 // section 2.2, where half the samples run dense and half at D = 64) take one
-// strided tensor-map pair each.  Within a segment, late query tiles come first
-// across all of its (b, h); a dilated segment whose dilated rows exceed a
-// quarter of L2 runs (b, h) by (b, h) instead, so that they stay in L2.
+// strided tensor-map pair each.  Within a dense segment, late query tiles come
+// first across all of its (b, h); a dilated segment runs (b, h) by (b, h),
+// late query tiles first, so that its dilated rows stay in L2.
 //
 // Two CTAs per SM, persistent over items blockIdx.x, +G, +2G, ... (G = grid
 // size = 2 x SMs; dense segments, the heaviest items, come first).  When a
@@ -133,7 +133,6 @@ struct Segment {
   int b_off;        // samples[b_off + i] is sample i; -1: sample i is b = i
   int8_t heads;     // kHeadsDense / kHeadsDil / kHeadsAll
   int8_t cls;       // -1: dense; c >= 0: dilation dil_D[c], tensor maps k[c], v[c]
-  int8_t bh_major;  // items (b, h) by (b, h) instead of query tile major
 };
 
 // Strided ("dilated") views of hk and hv, one pair per dilation class: row s
@@ -194,15 +193,13 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
     while (s + 1 < p.n_seg && idx >= p.seg[s + 1].begin) ++s;
     const Segment& g = p.seg[s];
     idx -= g.begin;
-    // Query tile major by default (late query tiles first across all of the
-    // segment's (b, h): the heaviest items first, and right after the scan
-    // the rows it left in L2 are read first).  A dilated segment whose
-    // dilated rows would not stay in L2 together goes (b, h) by (b, h), late
-    // query tiles first within each, so that the few (b, h) in flight keep
-    // theirs resident (7.6B hybrid layer: DRAM reads 2.18 -> 0.83 GB,
-    // 826 -> 787 us).
+    // dense segments: query tile major (the heaviest items, late query tiles,
+    // first across all of the segment's (b, h)); dilated segments: (b, h)
+    // major, late query tiles first within each (b, h), so that the few
+    // (b, h) in flight at a time keep their dilated rows in L2 (measured on
+    // the 7.6B hybrid layer: DRAM reads 2.18 -> 0.83 GB, 826 -> 787 us)
     int qi, bi, hi;
-    if (g.bh_major) {
+    if (g.cls >= 0) {
       const int pair = idx / p.NQ;
       qi = idx - pair * p.NQ;
       bi = pair / g.n_h;

@@ -334,10 +334,6 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
     Segment& g = p.seg[p.n_seg++];
     g.begin = (int)items; g.n_b = n_b; g.n_h = n_h; g.b_off = b_off;
     g.heads = (int8_t)heads; g.cls = (int8_t)cls;
-    // (b, h)-major items when the segment's dilated rows (k and v) exceed
-    // a quarter of the 126 MB L2
-    const long long dil_bytes = cls < 0 ? 0 : (long long)n_b * n_h * (T / p.dil_D[cls]) * 128 * 2 * 2;
-    g.bh_major = (int8_t)(dil_bytes > (32ll << 20));
     items += (long long)n_b * n_h * p.NQ;
   };
   if (Ds == nullptr) {
