@@ -135,28 +135,6 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return d;
 }
 
-// 2^x for a pair of values on the FMA pipe instead of the special-function
-// unit (which computes one exponential per lane every few cycles and limits a
-// softmax over 128 columns).  Range reduction: x = n + f with n = round(x)
-// (adding 1.5 * 2^23 rounds to an integer held in the low mantissa bits) and
-// f in [-0.5, 0.5]; 2^f is a cubic fitted here by a Remez exchange for least
-// maximum relative error on [-0.5, 0.5] (7.5e-5, far below the 2^-9 of a
-// bf16 result); the result's exponent field then gets n added.  Inputs below
-// -126 are clamped there (the result is then at most 2^-126 instead of 0;
-// -inf included); the caller never passes values above 2^8.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-  x.x = fmaxf(x.x, -126.f);
-  x.y = fmaxf(x.y, -126.f);
-  const float2 t = add2(x, make_float2(kRound, kRound));
-  const float2 f = sub2(x, sub2(t, make_float2(kRound, kRound)));
-  float2 p = fma2(f, make_float2(0.0551716685f, 0.0551716685f), make_float2(0.2426111251f, 0.2426111251f));
-  p = fma2(p, f, make_float2(0.6932609677f, 0.6932609677f));
-  p = fma2(p, f, make_float2(0.9999280572f, 0.9999280572f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
