@@ -503,6 +503,20 @@ int cache_layout(int B, int H, int Dh, int T_max, int D, int W, const uint8_t* h
   const long long target_ctas = (long long)sm_count() * kDecodeCtasPerSm;
   long long split = (keys_total + target_ctas - 1) / target_ctas;
   if (split < kMinSplitKeys) split = kMinSplitKeys;
+  // Keep every head's split count but even out its splits: the split becomes
+  // the largest per-split share among the heads, so no CTA streams more keys
+  // than it must (7.6B hybrid: 357 -> 347 keys, 24 and 6 splits per head).
+  {
+    long long even = kMinSplitKeys;
+    for (int h = 0; h < H; ++h) {
+      const bool dense = head_mask != nullptr && head_mask[h] != 0;
+      const long long keys = (dense ? T_max : T_max / D) + (dense ? 0 : W);
+      if (keys == 0) continue;
+      const long long n = (keys + split - 1) / split;
+      even = std::max(even, (keys + n - 1) / n);
+    }
+    split = std::min(split, even);
+  }
   if (split > (1 << 30)) split = 1 << 30;
   L->split_keys = (int)split;
   L->max_splits = (max_keys + L->split_keys - 1) / L->split_keys;
