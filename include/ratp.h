@@ -246,6 +246,21 @@ int ratp_dilated_attn_prefill_simt(const void* q, const void* hk, const void* hv
                                    int B, int T, int H, int Dh, int D, int W,
                                    const uint8_t* head_mask, int dtype, void* stream);
 
+/* Same computation as ratp_dilated_attn_prefill, with an optional workspace:
+ * device memory of at least RATP_ATTN_WORKSPACE_BYTES, 16-byte aligned, no
+ * initialisation needed (each call clears what it uses, on `stream`).  With
+ * it, a tensor-core launch that mixes dense and dilated work (a head_mask
+ * with dense heads and D > 1) hands its work items to CTAs as they become
+ * free instead of in fixed rounds, which balances items of very different
+ * cost; launches of one kind are unchanged.  NULL behaves as
+ * ratp_dilated_attn_prefill.  Calls sharing one workspace must be ordered on
+ * one stream.  Errors: as ratp_dilated_attn_prefill; ALIGN for a misaligned
+ * workspace. */
+#define RATP_ATTN_WORKSPACE_BYTES 256u
+int ratp_dilated_attn_prefill_ws(const void* q, const void* hk, const void* hv, void* o,
+                                 int B, int T, int H, int Dh, int D, int W,
+                                 const uint8_t* head_mask, int dtype, void* workspace, void* stream);
+
 /* ------------------------------------------------------------------------
  * Fused prefill: the recurrence of both streams and the dilated (+ windowed,
  * head-wise hybrid) attention over it in one launch (the full-sequence
@@ -300,6 +315,12 @@ int ratp_prefill_fused(const void* q, const void* xk, const void* xv, const void
 int ratp_dilated_attn_prefill_per_sample(const void* q, const void* hk, const void* hv, void* o,
                                          int B, int T, int H, int Dh, const int32_t* D_per_sample,
                                          int W, const uint8_t* head_mask, int dtype, void* stream);
+/* With the optional workspace of ratp_dilated_attn_prefill_ws (the same
+ * rules); a batch that mixes dense and dilated samples is dealt dynamically. */
+int ratp_dilated_attn_prefill_per_sample_ws(const void* q, const void* hk, const void* hv, void* o,
+                                            int B, int T, int H, int Dh, const int32_t* D_per_sample,
+                                            int W, const uint8_t* head_mask, int dtype, void* workspace,
+                                            void* stream);
 
 /* ------------------------------------------------------------------------
  * D-compressed KV cache and decode (RAT+ abstract: the KV cache shrinks by D).

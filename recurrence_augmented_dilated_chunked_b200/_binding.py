@@ -77,6 +77,8 @@ _SIGS = {
     "ratp_dilated_attn_prefill": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_simt": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P], _I),
     "ratp_dilated_attn_prefill_per_sample": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I, _P], _I),
+    "ratp_dilated_attn_prefill_ws": ([_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _P], _I),
+    "ratp_dilated_attn_prefill_per_sample_ws": ([_P, _P, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I, _P, _P], _I),
     "ratp_prefill_fused_workspace_bytes": ([_I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
     "ratp_prefill_fused": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _P, _SZ, _P], _I),
     "ratp_cache_bytes": ([_I, _I, _I, _I, _I, _I, _P, ctypes.POINTER(_SZ)], _I),
@@ -262,7 +264,27 @@ def scan_prefill_kv_noalloc(xk, xv, g, hk, hv, final_state=None):
     return hk, hv
 
 
-def _attn(fn_name, q, hk, hv, D, W, head_mask, out):
+ATTN_WORKSPACE_BYTES = 256
+_attn_ws_cache = {}
+
+
+def attn_workspace(device, stream=None) -> torch.Tensor:
+    """The attention's small device workspace for ``stream`` (default: the
+    device's current stream), cached per (device, stream): calls sharing one
+    must be ordered on one stream.  It needs no initialisation."""
+    device = torch.device(device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    key = (str(device), stream.cuda_stream)
+    with _lock:
+        ws = _attn_ws_cache.get(key)
+        if ws is None:
+            ws = torch.empty(ATTN_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+            _attn_ws_cache[key] = ws
+    return ws
+
+
+def _attn(fn_name, q, hk, hv, D, W, head_mask, out, workspace=False):
     lib = load_library()
     _need(q, "q")
     _need(hk, "hk", q.dtype)
@@ -272,15 +294,21 @@ def _attn(fn_name, q, hk, hv, D, W, head_mask, out):
         out = torch.empty_like(q)
     _need(out, "out", q.dtype)
     _buf, mp = _mask_buf(head_mask, H)
-    _check(fn_name, getattr(lib, fn_name)(
-        _ptr(q), _ptr(hk), _ptr(hv), _ptr(out), B, T, H, Dh, int(D), int(W), mp,
-        _DTYPE[q.dtype], _stream(q)))
+    args = [_ptr(q), _ptr(hk), _ptr(hv), _ptr(out), B, T, H, Dh, int(D), int(W), mp, _DTYPE[q.dtype]]
+    if workspace is not False:
+        args.append(_ptr(workspace) if workspace is not None else None)
+    _check(fn_name, getattr(lib, fn_name)(*args, _stream(q)))
     return out
 
 
-def dilated_attn_prefill(q, hk, hv, D, W=0, head_mask=None, out=None):
-    """Dilated (+ windowed) causal attention of q over recurrent hk, hv."""
-    return _attn("ratp_dilated_attn_prefill", q, hk, hv, D, W, head_mask, out)
+def dilated_attn_prefill(q, hk, hv, D, W=0, head_mask=None, out=None, workspace=None):
+    """Dilated (+ windowed) causal attention of q over recurrent hk, hv.
+    ``workspace``: an ``attn_workspace`` (default: the cached one of q's
+    device and current stream), with which launches that mix dense and
+    dilated items deal them dynamically."""
+    if workspace is None and q.is_cuda:
+        workspace = attn_workspace(q.device)
+    return _attn("ratp_dilated_attn_prefill_ws", q, hk, hv, D, W, head_mask, out, workspace)
 
 
 def dilated_attn_prefill_simt(q, hk, hv, D, W=0, head_mask=None, out=None):
@@ -288,9 +316,10 @@ def dilated_attn_prefill_simt(q, hk, hv, D, W=0, head_mask=None, out=None):
     return _attn("ratp_dilated_attn_prefill_simt", q, hk, hv, D, W, head_mask, out)
 
 
-def dilated_attn_prefill_per_sample(q, hk, hv, D_per_sample, W=0, head_mask=None, out=None):
+def dilated_attn_prefill_per_sample(q, hk, hv, D_per_sample, W=0, head_mask=None, out=None, workspace=None):
     """Dilated attention with one dilation per sample (``D_per_sample``: B
-    ints >= 1; 1 = the sample runs dense) in one launch; bf16, Dh = 128."""
+    ints >= 1; 1 = the sample runs dense) in one launch; bf16, Dh = 128.
+    ``workspace`` as for ``dilated_attn_prefill``."""
     lib = load_library()
     _need(q, "q")
     _need(hk, "hk", q.dtype)
@@ -308,9 +337,11 @@ def dilated_attn_prefill_per_sample(q, hk, hv, D_per_sample, W=0, head_mask=None
     mbuf, mp = _mask_buf(head_mask, H)
     if q.dtype not in _DTYPE:
         raise ValueError("unsupported dtype %s" % q.dtype)
-    _check("ratp_dilated_attn_prefill_per_sample", lib.ratp_dilated_attn_prefill_per_sample(
+    if workspace is None and q.is_cuda:
+        workspace = attn_workspace(q.device)
+    _check("ratp_dilated_attn_prefill_per_sample_ws", lib.ratp_dilated_attn_prefill_per_sample_ws(
         _ptr(q), _ptr(hk), _ptr(hv), _ptr(out), B, T, H, Dh, ctypes.cast(dbuf, ctypes.c_void_p),
-        int(W), mp, _DTYPE[q.dtype], _stream(q)))
+        int(W), mp, _DTYPE[q.dtype], _ptr(workspace) if workspace is not None else None, _stream(q)))
     return out
 
 

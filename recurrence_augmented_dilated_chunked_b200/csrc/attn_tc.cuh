@@ -38,7 +38,9 @@
 // ~D x), every other round is dealt in reverse CTA order, so that the CTAs
 // that drew the heaviest items in one round draw the lightest in the next
 // (7.6B hybrid layer: 797 -> 753 us; a single segment keeps plain rounds,
-// which measured 2.6% faster on an all-dense layer).  Per CTA, tensor memory holds S (64 columns), two P buffers (bf16
+// which measured 2.6% faster on an all-dense layer).  Given a workspace, a
+// mixed launch instead hands out items from a counter as CTAs become free
+// (p.dynamic, through the same item ring as the fused prefill).  Per CTA, tensor memory holds S (64 columns), two P buffers (bf16
 // pairs, 32 columns each) and O (128 columns): 256 columns, half an SM's.
 // Because S and P are separate, S = Q K^T of tile n+1 is issued as soon as
 // the softmax has read S of tile n, so the tensor core computes the next
@@ -133,6 +135,7 @@ struct Segment {
   int b_off;        // samples[b_off + i] is sample i; -1: sample i is b = i
   int8_t heads;     // kHeadsDense / kHeadsDil / kHeadsAll
   int8_t cls;       // -1: dense; c >= 0: dilation dil_D[c], tensor maps k[c], v[c]
+  int tail;         // dilated: (b, h) pairs from this one on are interleaved
 };
 
 // Strided ("dilated") views of hk and hv, one pair per dilation class: row s
@@ -147,6 +150,7 @@ struct Params {
   int B, T, H, W_eff, NQ;
   int n_items, n_seg, n_cls;
   int alternate;          // deal every other round of items in reverse CTA order
+  int dynamic;            // items drawn from the counter ctl.items (workspace given, mixed segments)
   float scale_log2;
   int o_align32;          // output base 32-byte aligned (rows are 256 bytes)
   int dil_D[kMaxDil];
@@ -198,10 +202,21 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
     // major, late query tiles first within each (b, h), so that the few
     // (b, h) in flight at a time keep their dilated rows in L2 (measured on
     // the 7.6B hybrid layer: DRAM reads 2.18 -> 0.83 GB, 826 -> 787 us)
+    // With dynamic dealing the last (b, h) pairs of a dilated segment (from
+    // g.tail on) are interleaved, late query tiles first across them, so that
+    // the launch ends on light items (fewer than 32 pairs' rows in flight).
     int qi, bi, hi;
     if (g.cls >= 0) {
-      const int pair = idx / p.NQ;
-      qi = idx - pair * p.NQ;
+      int pair;
+      if (idx < g.tail * p.NQ) {
+        pair = idx / p.NQ;
+        qi = idx - pair * p.NQ;
+      } else {
+        const int j = idx - g.tail * p.NQ;
+        const int n_t = g.n_b * g.n_h - g.tail;
+        qi = j / n_t;
+        pair = g.tail + (j - qi * n_t);
+      }
       bi = pair / g.n_h;
       hi = pair - bi * g.n_h;
     } else {
@@ -376,9 +391,10 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       __syncthreads();
     }
   }
-  // This CTA's items: FUSED draws them one by one from the launch's item
-  // counter (ascending), the producer passing each index on through the ring
-  // (an index >= n_items ends the loop); otherwise blockIdx.x, +G, +2G, ...
+  // This CTA's items: FUSED (and a launch with p.dynamic) draws them one by
+  // one from the launch's item counter, the producer passing each index on
+  // through the ring (an index >= n_items ends the loop); otherwise
+  // blockIdx.x, +G, +2G, ... (every other round reversed with p.alternate).
   // The producer runs at most a few items ahead of the MMA issuer and the
   // softmax (it waits for O += P V of tile n-2 before it loads tile n), far
   // less than the ring's depth.
@@ -387,7 +403,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     return (p.alternate && (li & 1)) ? (li + 1) * G - 1 - c : c + li * G;
   };
   auto item_at = [&](int li) -> int {
-    if (!FUSED) return item_of(li);
+    if (!FUSED && !p.dynamic) return item_of(li);
     if (!mbar_wait(b_item + 8 * (li % kItemRing), (uint32_t)(li / kItemRing) & 1u, s_abort)) return -1;
     return s_items[li % kItemRing];
   };
@@ -404,7 +420,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     for (int li = 0;; ++li) {
       int idx;
-      if (FUSED) {
+      if (FUSED || p.dynamic) {
         if (lane == 0) {
           idx = ok ? (int)min(atomicAdd(p.ctl.items, 1u), (unsigned int)p.n_items) : p.n_items;
           s_items[li % kItemRing] = idx;           // n_items: no more items

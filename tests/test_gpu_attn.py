@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import recurrence_augmented_dilated_chunked_b200 as ratp
-from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, prefill_inputs
+from recurrence_augmented_dilated_chunked_b200 import WORKLOADS, _binding, prefill_inputs
 from parity import assert_close, bits_equal, to64
 
 pytestmark = pytest.mark.gpu
@@ -183,3 +183,24 @@ def test_small_shape_sweep(Dh, dtype, D):
             n += 1
     ratp.last_error()
     assert n >= 10
+
+
+@pytest.mark.parametrize("B,T,H,D,W,dense", [(2, 700, 4, 4, 0, (0, 1)), (1, 1100, 2, 64, 128, (1,)),
+                                             (1, 130, 256, 2, 3, tuple(range(0, 256, 7))),
+                                             (4, 1024, 40, 4, 0, (0, 1))])
+def test_mixed_launch_dynamic_and_static_dealing_agree_bitwise(B, T, H, D, W, dense):
+    """A launch that mixes dense and dilated items deals them dynamically when
+    given a workspace (the binding's default) and in fixed rounds without one
+    (ratp_dilated_attn_prefill); every item is computed the same way whichever
+    CTA takes it, so the outputs are bit-identical, and the static one matches
+    the oracle.  The last case has more than 32 dilated (b, h), so its tail is
+    interleaved."""
+    q, k, v = (t.to(DEV) for t in _qkv(B, T, H, 128, "bf16", seed=5 * T + D, qscale=2.0))
+    mask = [1 if h in dense else 0 for h in range(H)]
+    o_dyn = ratp.dilated_attn_prefill(q, k, v, D, W, head_mask=mask)
+    o_static = _binding._attn("ratp_dilated_attn_prefill", q, k, v, D, W, mask, None)
+    ratp.last_error()
+    assert torch.equal(o_dyn, o_static)
+    if B * T * H <= 2 * 700 * 4:
+        ref = oracle.attention(to64(q.cpu()), to64(k.cpu()), to64(v.cpu()), D, W, dense_mask=mask)
+        assert_close(o_static, ref, "bf16", "static dealing")

@@ -107,3 +107,24 @@ def test_per_sample_largest_batch():
     with pytest.raises(RatpError) as e:
         ratp.dilated_attn_prefill_per_sample(q2, hk2, hv2, [1] * (B + 1))
     assert e.value.code == 2
+
+
+def test_per_sample_dynamic_and_static_dealing_agree_bitwise():
+    """With the binding's workspace the mixed batch is dealt dynamically;
+    without one (the plain C entry point), in fixed rounds: same bits."""
+    import ctypes
+    from recurrence_augmented_dilated_chunked_b200 import _binding
+    Ds = [1, 64, 1, 64, 4, 1]
+    B, T, H = len(Ds), 900, 3
+    q, hk, hv = _inputs(B, T, H, seed=44)
+    o_dyn = ratp.dilated_attn_prefill_per_sample(q, hk, hv, Ds, 16, head_mask=[0, 1, 0])
+    o_static = torch.empty_like(q)
+    lib = _binding.load_library()
+    dbuf = (ctypes.c_int32 * B)(*Ds)
+    mbuf, mp = _binding._mask_buf([0, 1, 0], H)
+    rc = lib.ratp_dilated_attn_prefill_per_sample(
+        _binding._ptr(q), _binding._ptr(hk), _binding._ptr(hv), _binding._ptr(o_static), B, T, H, 128,
+        ctypes.cast(dbuf, ctypes.c_void_p), 16, mp, 1, _binding._stream(q))
+    assert rc == 0
+    ratp.last_error()
+    assert bits_equal(o_dyn, o_static)
