@@ -40,7 +40,7 @@
 // (7.6B hybrid layer: 797 -> 753 us; a single segment keeps plain rounds,
 // which measured 2.6% faster on an all-dense layer).  Given a workspace, a
 // mixed launch instead hands out items from a counter as CTAs become free
-// (p.dynamic, through the same item ring as the fused prefill).  Per CTA, tensor memory holds S (64 columns), two P buffers (bf16
+// (attn_kernel<false, true>, through the same item ring as the fused prefill).  Per CTA, tensor memory holds S (64 columns), two P buffers (bf16
 // pairs, 32 columns each) and O (128 columns): 256 columns, half an SM's.
 // Because S and P are separate, S = Q K^T of tile n+1 is issued as soon as
 // the softmax has read S of tile n, so the tensor core computes the next
@@ -150,7 +150,6 @@ struct Params {
   int B, T, H, W_eff, NQ;
   int n_items, n_seg, n_cls;
   int alternate;          // deal every other round of items in reverse CTA order
-  int dynamic;            // items drawn from the counter ctl.items (workspace given, mixed segments)
   float scale_log2;
   int o_align32;          // output base 32-byte aligned (rows are 256 bytes)
   int dil_D[kMaxDil];
@@ -178,7 +177,7 @@ struct Item {
   bool dense;
 };
 
-template <bool FUSED>
+template <bool FUSED, bool DYN>
 __device__ __forceinline__ Item make_item(const Params& p, int idx) {
   Item it;
   if (FUSED) {
@@ -202,13 +201,13 @@ __device__ __forceinline__ Item make_item(const Params& p, int idx) {
     // major, late query tiles first within each (b, h), so that the few
     // (b, h) in flight at a time keep their dilated rows in L2 (measured on
     // the 7.6B hybrid layer: DRAM reads 2.18 -> 0.83 GB, 826 -> 787 us)
-    // With dynamic dealing the last (b, h) pairs of a dilated segment (from
-    // g.tail on) are interleaved, late query tiles first across them, so that
-    // the launch ends on light items (fewer than 32 pairs' rows in flight).
+    // With dynamic dealing (DYN) the last (b, h) pairs of a dilated segment
+    // (from g.tail on) are interleaved, late query tiles first across them, so
+    // that the launch ends on light items (at most 32 pairs' rows in flight).
     int qi, bi, hi;
     if (g.cls >= 0) {
       int pair;
-      if (idx < g.tail * p.NQ) {
+      if (!DYN || idx < g.tail * p.NQ) {
         pair = idx / p.NQ;
         qi = idx - pair * p.NQ;
       } else {
@@ -304,7 +303,11 @@ __device__ __forceinline__ bool wait_chunks(const Params& p, const Item& it, uns
   return true;
 }
 
-template <bool FUSED>
+// DYN: a mixed non-fused launch given a workspace; its items are drawn from
+// the counter ctl.items (a separate instance, so that the static kernel's
+// code is unchanged: the larger body cost the static path instruction
+// fetches, T=16K +4% cycles).
+template <bool FUSED, bool DYN = false>
 __global__ void __launch_bounds__(FUSED ? kThreadsFused : kThreads, kCtasPerSm)
 attn_kernel(const __grid_constant__ CUtensorMap tm_q,
             const __grid_constant__ CUtensorMap tm_kpos,
@@ -391,7 +394,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       __syncthreads();
     }
   }
-  // This CTA's items: FUSED (and a launch with p.dynamic) draws them one by
+  // This CTA's items: FUSED (and a DYN launch) draws them one by
   // one from the launch's item counter, the producer passing each index on
   // through the ring (an index >= n_items ends the loop); otherwise
   // blockIdx.x, +G, +2G, ... (every other round reversed with p.alternate).
@@ -403,7 +406,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     return (p.alternate && (li & 1)) ? (li + 1) * G - 1 - c : c + li * G;
   };
   auto item_at = [&](int li) -> int {
-    if (!FUSED && !p.dynamic) return item_of(li);
+    if (!FUSED && !DYN) return item_of(li);
     if (!mbar_wait(b_item + 8 * (li % kItemRing), (uint32_t)(li / kItemRing) & 1u, s_abort)) return -1;
     return s_items[li % kItemRing];
   };
@@ -420,7 +423,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
     bool ok = true;
     for (int li = 0;; ++li) {
       int idx;
-      if (FUSED || p.dynamic) {
+      if (FUSED || DYN) {
         if (lane == 0) {
           idx = ok ? (int)min(atomicAdd(p.ctl.items, 1u), (unsigned int)p.n_items) : p.n_items;
           s_items[li % kItemRing] = idx;           // n_items: no more items
@@ -431,7 +434,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         idx = item_of(li);
       }
       if (!ok || idx >= p.n_items) break;
-      const Item it = make_item<FUSED>(p, idx);
+      const Item it = make_item<FUSED, DYN>(p, idx);
       if (FUSED && !wait_chunks(p, it, tag, lane, s_abort)) ok = false;
       if (ok && lane == 0) {
         for (int j = 0; j < it.n_tiles; ++j, ++n) {
@@ -523,7 +526,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int idx = item_at(li);
         if (idx < 0) { ok = false; break; }
         if (idx >= p.n_items) break;
-        const int n_tiles = make_item<FUSED>(p, idx).n_tiles;
+        const int n_tiles = make_item<FUSED, DYN>(p, idx).n_tiles;
         if (!mbar_wait(b_qfull, li & 1, s_abort)) { ok = false; break; }
         if (!issue_s(n)) { ok = false; break; }
         for (int j = 1; j < n_tiles; ++j) {
@@ -554,7 +557,7 @@ attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int idx = item_at(li);
       if (!warp_all(idx >= 0)) { ok = false; break; }
       if (idx >= p.n_items) break;
-      const Item it = make_item<FUSED>(p, idx);
+      const Item it = make_item<FUSED, DYN>(p, idx);
       const int t = it.t0 + r;
       const int lim_dil = it.dense ? (t + 1) : (max(0, t - p.W_eff + 1) / it.Dd);
       const int w_lo = max(t - p.W_eff + 1, 0);

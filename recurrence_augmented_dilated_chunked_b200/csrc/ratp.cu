@@ -370,8 +370,8 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
   // 32 (b, h) pairs of each dilated segment are interleaved so that the launch
   // ends on light items.  A single segment keeps static dealing (dynamic
   // dealing measured 1-8% slower there).
-  if (ws != nullptr && p.n_seg > 1) {
-    p.dynamic = 1;
+  const bool dynamic = ws != nullptr && p.n_seg > 1;
+  if (dynamic) {
     p.ctl.items = static_cast<unsigned int*>(ws);
     for (int i = 0; i < p.n_seg; ++i) {
       Segment& g = p.seg[i];
@@ -403,7 +403,7 @@ int launch_attn_tc(const void* q, const void* hk, const void* hv, void* o,
   }
   attn_tc::ScanMaps sm_unused;
   memset(&sm_unused, 0, sizeof(sm_unused));
-  auto kernel = attn_tc::attn_kernel<false>;
+  auto kernel = dynamic ? attn_tc::attn_kernel<false, true> : attn_tc::attn_kernel<false, false>;
   if (!ensure_smem(kernel, (int)attn_tc::kSmemBytes)) return RATP_ERR_CUDA;
   const int slots = attn_tc::kCtasPerSm * sm_count();
   const int grid = p.n_items < slots ? p.n_items : slots;
