@@ -10,6 +10,7 @@ package is the thin ctypes binding plus the seeded input generators.
 from ._binding import (  # noqa: F401
     KVCache,
     RatpError,
+    attn_workspace,
     dilated_attn_prefill,
     dilated_attn_prefill_per_sample,
     dilated_attn_prefill_simt,
