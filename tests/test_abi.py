@@ -120,6 +120,21 @@ def test_fused_prefill_rejects_bad_arguments_on_host(lib):
     assert lib.ratp_prefill_fused(p, p, p, p, p, p, p, None, 1, 8, 1, 128, 4, -1, None, 1, ws, 1 << 20, None) == 1
 
 
+def test_attention_workspace_entry_points_check_arguments_on_host(lib):
+    p = ctypes.c_void_p(16)
+    # a misaligned workspace, then the checks of the plain calls (D < 1, W < 0)
+    assert lib.ratp_dilated_attn_prefill_ws(p, p, p, p, 1, 8, 1, 128, 4, 0, None, 1,
+                                            ctypes.c_void_p(18), None) == 3
+    assert lib.ratp_dilated_attn_prefill_ws(p, p, p, p, 1, 8, 1, 128, 0, 0, None, 1, p, None) == 1
+    assert lib.ratp_dilated_attn_prefill_ws(p, p, p, p, 1, 8, 1, 128, 4, -1, None, 1, p, None) == 1
+    ds = (ctypes.c_int32 * 2)(1, 0)
+    assert lib.ratp_dilated_attn_prefill_per_sample_ws(p, p, p, p, 2, 8, 1, 128, ctypes.cast(ds, ctypes.c_void_p),
+                                                       0, None, 1, p, None) == 1
+    assert lib.ratp_dilated_attn_prefill_per_sample_ws(p, p, p, p, 2, 8, 1, 128, ctypes.cast(ds, ctypes.c_void_p),
+                                                       0, None, 1, ctypes.c_void_p(18), None) == 3
+    assert _binding.ATTN_WORKSPACE_BYTES == 256
+
+
 def test_cache_bytes_query(lib):
     n = ctypes.c_size_t()
     assert lib.ratp_cache_bytes(64, 16, 128, 33024, 64, 128, None, ctypes.byref(n)) == 0
